@@ -1,0 +1,227 @@
+// merge.cu -- LSE-weighted merge of attention states under a reuse mask, with fused
+// partition importance, plus the stand-alone importance kernel and the reduction that
+// turns per-block importance sums into means.
+//
+// Math (DiTango web summary, Methodology 2 "State Composition": output and log-sum-exp
+// states compose associatively and commutatively; Methodology 1: fresh or reused per
+// group, importance refreshed at anchor steps):
+//   LSE(i) = ln sum_p exp(LSE_p(i)),   O(i) = sum_p exp(LSE_p(i) - LSE(i)) O_p(i),
+//   w[qg][p] = mean over b, h, rows i of qg of exp(LSE_p(i) - LSE(i)),
+// where the state of partition p is the fresh one when fresh[qg][p / G], else the cached.
+//
+// The merge is bound by HBM reads of the P states per row.  A block owns 128 rows of one
+// query group of one (b, h):
+//   phase 1  one thread per row reads the P log-sum-exps (coalesced across rows), forms
+//            LSE with a running max, writes LSE and the P weights to shared memory;
+//   phase 2  one warp per row streams the P state rows with 128-bit loads, 2..4 states
+//            per warp iteration (a state row is D * elem bytes = 128..512 bytes), 8
+//            iterations in flight, and reduces the partial sums with shuffles.
+// Per-block importance sums go to a workspace [block][P]; reduce_w_kernel adds them per
+// query group in a fixed order (deterministic) and divides by the row count.
+#include "pa_device.cuh"
+#include "pa_launch.h"
+
+namespace pa {
+namespace {
+
+constexpr int kMR = 128;            // rows per block = threads per block
+constexpr int kUnroll = 8;          // state loads in flight per lane
+
+__device__ __forceinline__ int find_group(const int* start, int n, int x) {
+  int g = 0;
+  while (g + 1 < n && start[g + 1] <= x) ++g;
+  return g;
+}
+
+template <typename T> struct Acc;
+template <> struct Acc<float> {
+  static constexpr int E = 4;
+  __device__ static void add(float (&a)[8], const uint4& v, float w) {
+    a[0] = fmaf(w, __uint_as_float(v.x), a[0]);
+    a[1] = fmaf(w, __uint_as_float(v.y), a[1]);
+    a[2] = fmaf(w, __uint_as_float(v.z), a[2]);
+    a[3] = fmaf(w, __uint_as_float(v.w), a[3]);
+  }
+  __device__ static uint4 pack(const float (&a)[8]) {
+    return make_uint4(__float_as_uint(a[0]), __float_as_uint(a[1]), __float_as_uint(a[2]),
+                      __float_as_uint(a[3]));
+  }
+};
+template <> struct Acc<__nv_bfloat16> {
+  static constexpr int E = 8;
+  __device__ static void add2(float& a0, float& a1, uint32_t u, float w) {
+    a0 = fmaf(w, __uint_as_float(u << 16), a0);
+    a1 = fmaf(w, __uint_as_float(u & 0xFFFF0000u), a1);
+  }
+  __device__ static void add(float (&a)[8], const uint4& v, float w) {
+    add2(a[0], a[1], v.x, w);
+    add2(a[2], a[3], v.y, w);
+    add2(a[4], a[5], v.z, w);
+    add2(a[6], a[7], v.w, w);
+  }
+  __device__ static uint4 pack(const float (&a)[8]) {
+    return make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                      pack_bf16x2(a[6], a[7]));
+  }
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kMR) merge_kernel(const __grid_constant__ MergeParams prm) {
+  extern __shared__ float sW[];                    // [P][kMR + 1] merged weights
+  constexpr int kRowBytes = D * sizeof(T);
+  constexpr int LPR = kRowBytes / 16;              // lanes per state row
+  constexpr int SPW = 32 / LPR;                    // state rows per warp iteration
+  const int P = prm.P;
+  const int bh = blockIdx.x / prm.blocks_per_bh;
+  const int blk = blockIdx.x - bh * prm.blocks_per_bh;
+  const int qg = find_group(prm.blk_start, prm.QG, blk);
+  const int r0 = prm.qg_row0[qg] + (blk - prm.blk_start[qg]) * kMR;
+  const int nrows = min(kMR, prm.qg_row0[qg + 1] - r0);
+  const size_t BHN = static_cast<size_t>(prm.BH) * prm.N;
+  const size_t hrow0 = static_cast<size_t>(bh) * prm.N + r0;
+
+  // ---- phase 1: LSE and weights, one thread per row
+  {
+    const int t = threadIdx.x;
+    const bool ok = t < nrows;
+    float m = -INFINITY, l = 0.0f;
+    if (ok) {
+      for (int p = 0; p < P; ++p) {
+        const float* src = fresh_bit(prm.fresh_bits, qg, p) ? prm.lse_fresh : prm.lse_cached;
+        const float L = src[p * BHN + hrow0 + t];
+        if (L > m) {
+          l = l * expf(m - L) + 1.0f;
+          m = L;
+        } else if (L > -INFINITY) {
+          l += expf(L - m);
+        }
+      }
+    }
+    const float lse = m > -INFINITY ? m + logf(l) : -INFINITY;
+    if (ok) prm.lse[hrow0 + t] = lse;
+    for (int p = 0; p < P; ++p) {
+      float w = 0.0f;
+      if (ok && lse > -INFINITY) {
+        const float* src = fresh_bit(prm.fresh_bits, qg, p) ? prm.lse_fresh : prm.lse_cached;
+        w = expf(src[p * BHN + hrow0 + t] - lse);
+      }
+      sW[p * (kMR + 1) + t] = w;
+    }
+  }
+  __syncthreads();
+  if (prm.w_partial) {
+    for (int p = threadIdx.x; p < P; p += kMR) {
+      float s = 0.0f;
+      for (int i = 0; i < nrows; ++i) s += sW[p * (kMR + 1) + i];
+      prm.w_partial[static_cast<size_t>(blockIdx.x) * P + p] = s;
+    }
+  }
+
+  // ---- phase 2: weighted sum of the state rows, one warp per row
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane % LPR, slot = lane / LPR;
+  const uint8_t* of = static_cast<const uint8_t*>(prm.o_fresh);
+  const uint8_t* oc = static_cast<const uint8_t*>(prm.o_cached);
+  for (int i = warp; i < nrows; i += kMR / 32) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const size_t rowoff = (hrow0 + i) * kRowBytes + sub * 16;
+    for (int p0 = 0; p0 < P; p0 += SPW * kUnroll) {
+      uint4 v[kUnroll];
+      float wt[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int p = p0 + u * SPW + slot;
+        wt[u] = 0.0f;
+        v[u] = make_uint4(0, 0, 0, 0);
+        if (p < P) {
+          wt[u] = sW[p * (kMR + 1) + i];
+          const uint8_t* base = fresh_bit(prm.fresh_bits, qg, p) ? of : oc;
+          v[u] = __ldg(reinterpret_cast<const uint4*>(base + p * BHN * kRowBytes + rowoff));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) Acc<T>::add(acc, v[u], wt[u]);
+    }
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1)
+#pragma unroll
+      for (int e = 0; e < Acc<T>::E; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    if (slot == 0)
+      *reinterpret_cast<uint4*>(static_cast<uint8_t*>(prm.o) + rowoff) = Acc<T>::pack(acc);
+  }
+}
+
+__global__ void __launch_bounds__(kMR) importance_kernel(const __grid_constant__ ImportanceParams prm) {
+  __shared__ float sPart[kMR / 32][PA_MAX_P];
+  const int P = prm.P;
+  const int bh = blockIdx.x / prm.blocks_per_bh;
+  const int blk = blockIdx.x - bh * prm.blocks_per_bh;
+  const int qg = find_group(prm.blk_start, prm.QG, blk);
+  const int r0 = prm.qg_row0[qg] + (blk - prm.blk_start[qg]) * kMR;
+  const int nrows = min(kMR, prm.qg_row0[qg + 1] - r0);
+  const size_t BHN = static_cast<size_t>(prm.BH) * prm.N;
+  const size_t hrow = static_cast<size_t>(bh) * prm.N + r0 + threadIdx.x;
+  const bool ok = static_cast<int>(threadIdx.x) < nrows;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float L = ok ? prm.lse[hrow] : -INFINITY;
+  for (int p = 0; p < P; ++p) {
+    float w = (ok && L > -INFINITY) ? expf(prm.lse_part[p * BHN + hrow] - L) : 0.0f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) w += __shfl_xor_sync(0xffffffffu, w, off);
+    if (lane == 0) sPart[warp][p] = w;
+  }
+  __syncthreads();
+  for (int p = threadIdx.x; p < P; p += kMR) {
+    float s = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kMR / 32; ++w) s += sPart[w][p];
+    prm.w_partial[static_cast<size_t>(blockIdx.x) * P + p] = s;
+  }
+}
+
+__global__ void __launch_bounds__(128) reduce_w_kernel(const __grid_constant__ ReduceWParams prm) {
+  const int qg = blockIdx.x;
+  const int b0 = prm.blk_start[qg], b1 = prm.blk_start[qg + 1];
+  for (int p = threadIdx.x; p < prm.P; p += blockDim.x) {
+    double s = 0.0;
+    for (int bh = 0; bh < prm.BH; ++bh)
+      for (int b = b0; b < b1; ++b)
+        s += prm.w_partial[(static_cast<size_t>(bh) * prm.blocks_per_bh + b) * prm.P + p];
+    prm.w[qg * prm.P + p] = static_cast<float>(s * prm.inv_count[qg]);
+  }
+}
+
+template <typename T, int D>
+int merge_impl(const MergeParams& prm, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(prm.P) * (kMR + 1) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(merge_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  const long long blocks = static_cast<long long>(prm.BH) * prm.blocks_per_bh;
+  merge_kernel<T, D><<<static_cast<unsigned>(blocks), kMR, smem, st>>>(prm);
+  return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace
+
+int merge_rows_per_block() { return kMR; }
+
+int launch_merge(const MergeParams& prm, int dtype, cudaStream_t st) {
+  if (dtype == PA_BF16) return prm.D == 64 ? merge_impl<__nv_bfloat16, 64>(prm, st) : merge_impl<__nv_bfloat16, 128>(prm, st);
+  return prm.D == 64 ? merge_impl<float, 64>(prm, st) : merge_impl<float, 128>(prm, st);
+}
+
+int launch_importance(const ImportanceParams& prm, cudaStream_t st) {
+  const long long blocks = static_cast<long long>(prm.BH) * prm.blocks_per_bh;
+  importance_kernel<<<static_cast<unsigned>(blocks), kMR, 0, st>>>(prm);
+  return static_cast<int>(cudaGetLastError());
+}
+
+int launch_reduce_w(const ReduceWParams& prm, cudaStream_t st) {
+  reduce_w_kernel<<<prm.QG, 128, 0, st>>>(prm);
+  return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace pa

@@ -1,0 +1,25 @@
+// pa_launch.h -- host-side launchers of libpa's kernels (internal; the public ABI is pa.h).
+// Each returns a cudaError_t value (0 on success).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+int launch_attn_tc(const TcParams& prm, int units, cudaStream_t st);
+int attn_tc_tile_rows();
+
+int launch_attn_f32(const F32AttnParams& prm, cudaStream_t st);
+int attn_f32_tile_rows();
+
+int launch_merge(const MergeParams& prm, int dtype, cudaStream_t st);
+int merge_rows_per_block();
+int launch_importance(const ImportanceParams& prm, cudaStream_t st);
+int launch_reduce_w(const ReduceWParams& prm, cudaStream_t st);
+
+int launch_relayout(const void* src, void* dst, long long n0, long long n1, int N, int H,
+                    int row_bytes, int sm_count, cudaStream_t st);
+
+}  // namespace pa

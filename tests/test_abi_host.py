@@ -1,0 +1,80 @@
+"""CPU tests of the C ABI library and the host-side logic (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+import sequence_partition_attn_b200 as pa
+from sequence_partition_attn_b200 import build as pa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pa_build.build()
+    return pa.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "pa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(pa_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_documented_entry_points():
+    assert set(header_functions()) == set(pa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {pa.lib_path()}").read()
+    for name in header_functions():
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+def test_library_is_built_for_sm100a_only(lib):
+    flags = " ".join(pa_build.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+    assert flags.count("-gencode") == 1
+
+
+def test_version_and_init_without_device(lib):
+    assert lib.pa_version().decode().startswith("libpa")
+    ctx = ctypes.c_void_p()
+    rc = lib.pa_init(0, ctypes.byref(ctx))
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:
+        has_gpu = False
+    if not has_gpu:
+        assert rc in (-1, -3, -5)           # no device: an error code, never a crash
+        assert not ctx.value
+        assert lib.pa_last_error(None)
+    else:
+        lib.pa_destroy(ctx)
+
+
+def test_null_context_is_rejected(lib):
+    assert lib.pa_partition_attn(None, None, None) == -1
+    assert lib.pa_merge_states(None, None, None) == -1
+    assert lib.pa_importance(None, 1, 1, 1, 1, 1, None, None, None, None, None) == -1
+    assert lib.pa_relayout_seq2head(None, None, None, 1, 1, 8, 2, 1, -1, None) == -1
+    assert lib.pa_sync_status(None, None) == -1
+    assert b"ctx" in lib.pa_last_error(None)
+    lib.pa_destroy(None)                   # no-op
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_host_reuse_selection_matches_the_oracle(seed):
+    rng = np.random.default_rng(seed)
+    QG, P = rng.integers(1, 9), rng.integers(1, 33)
+    G = int(rng.integers(1, P + 1))
+    QG = -(-P // G)
+    w = rng.dirichlet(np.ones(P), size=QG) * rng.uniform(0.2, 1.5)
+    w[rng.random(w.shape) < 0.2] = 0.05                 # exact threshold hits
+    np.testing.assert_array_equal(pa.select_fresh(w, G, 0.05), O.select_fresh(w, G, 0.05))

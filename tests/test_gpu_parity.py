@@ -1,0 +1,229 @@
+"""GPU parity: every libpa entry point, through the C ABI, against the fp64 oracle on the
+same seeded inputs, at oracle-sized shapes that span several tiles and ragged tails."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from tests.helpers import TOL, compare_states, maxerr, run_reuse_case
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pa():
+    from sequence_partition_attn_b200 import build
+    build.build()
+    import sequence_partition_attn_b200 as m
+    return m
+
+
+@pytest.fixture(scope="module")
+def ctx(pa):
+    c = pa.Context(0)
+    yield c
+    c.close()
+
+
+DEV = "cuda:0"
+
+
+# --------------------------------------------------------------------------- relayout
+@pytest.mark.parametrize("N,H,D,dt,chunks", [(1000, 3, 128, torch.bfloat16, 16),
+                                               (777, 5, 64, torch.float32, 3),
+                                               (64, 1, 8, torch.bfloat16, 1),
+                                               (7200 * 2, 24, 128, torch.bfloat16, 16)])
+def test_relayout_bit_exact(pa, ctx, N, H, D, dt, chunks):
+    g = torch.Generator().manual_seed(N + H)
+    src = torch.randn(N, H, D, generator=g).to(dt)
+    bits = torch.int16 if dt == torch.bfloat16 else torch.int32
+    ref = O.relayout_seq2head(src.view(bits).numpy(), chunks)
+    s = src.to(DEV)
+    dst = torch.full((H, N, D), float("nan"), dtype=dt, device=DEV)
+    for c in range(chunks):                       # chunk by chunk
+        pa.pa_relayout_seq2head(ctx, s, dst, n_chunks=chunks, chunk=c)
+    ctx.sync_status()
+    assert np.array_equal(dst.cpu().view(bits).numpy(), ref)
+    dst2 = torch.zeros_like(dst)
+    pa.pa_relayout_seq2head(ctx, s, dst2, n_chunks=chunks, chunk=-1)   # all at once
+    ctx.sync_status()
+    assert np.array_equal(dst2.cpu().view(bits).numpy(), ref)
+
+
+def test_relayout_single_chunk_touches_only_its_rows(pa, ctx):
+    N, H, D = 1000, 2, 64
+    src = torch.randn(N, H, D).to(torch.bfloat16).to(DEV)
+    dst = torch.zeros(H, N, D, dtype=torch.bfloat16, device=DEV)
+    pa.pa_relayout_seq2head(ctx, src, dst, n_chunks=4, chunk=2)    # rows [500, 750)
+    ctx.sync_status()
+    d = dst.cpu().float().numpy()
+    s = src.cpu().float().numpy()
+    assert np.array_equal(d[:, 500:750], s[500:750].transpose(1, 0, 2))
+    assert not d[:, :500].any() and not d[:, 750:].any()
+
+
+# --------------------------------------------------------------------------- merge / importance
+def _gen_states(seed, P, B, H, N, D, dt, empty=()):
+    rng = np.random.default_rng(seed)
+    lse = rng.normal(loc=3.0, scale=2.5, size=(P, B, H, N)).astype(np.float32)
+    o = rng.standard_normal((P, B, H, N, D)).astype(np.float32)
+    for p in empty:
+        lse[p] = -np.inf
+        o[p] = 0.0
+    o_t = torch.from_numpy(o).to(dt)
+    return o_t, torch.from_numpy(lse)
+
+
+@pytest.mark.parametrize("dt,D,N,P,G,B,H", [
+    (torch.bfloat16, 128, 1000, 8, 1, 1, 3),
+    (torch.bfloat16, 128, 2900, 32, 4, 1, 2),
+    (torch.bfloat16, 64, 517, 5, 2, 2, 2),
+    (torch.float32, 64, 1024, 4, 1, 1, 2),
+    (torch.float32, 128, 300, 64, 8, 1, 1),
+    (torch.bfloat16, 128, 640, 128, 16, 1, 1),
+])
+def test_merge_with_reuse_and_fused_importance(pa, ctx, dt, D, N, P, G, B, H):
+    off = W.part_offsets(N, P)
+    QG = -(-P // G)
+    rng = np.random.default_rng(N + P)
+    fresh = (rng.random((QG, QG)) < 0.4).astype(np.uint8)
+    empty = [p for p in range(P) if off[p + 1] == off[p]]
+    of, lf = _gen_states(1, P, B, H, N, D, dt, empty)
+    oc, lc = _gen_states(2, P, B, H, N, D, dt, empty)
+    o = torch.empty(B, H, N, D, dtype=dt, device=DEV)
+    lse = torch.empty(B, H, N, device=DEV)
+    w = torch.empty(QG, P, device=DEV)
+    pa.pa_merge_states(ctx, off, G, fresh, of.to(DEV), lf.to(DEV), oc.to(DEV), lc.to(DEV), o, lse, w)
+    ctx.sync_status()
+    f64 = lambda x: x.double().numpy()   # noqa: E731
+    ro, rl, ch = O.merge_with_reuse(f64(of), f64(lf), f64(oc), f64(lc), off, G, fresh)
+    rw = O.importance(ch, rl, off, G)
+    tol = TOL["bf16" if dt == torch.bfloat16 else "f32"]
+    # stored states are exact inputs; only the merge arithmetic and output rounding differ
+    o_tol = 1e-2 if dt == torch.bfloat16 else 1e-5
+    assert maxerr(o.float().cpu().numpy(), ro) <= o_tol
+    assert maxerr(lse.cpu().numpy(), rl) <= 1e-5 + 1e-6 * np.abs(rl).max()
+    assert maxerr(w.cpu().numpy(), rw) <= tol["w"]
+
+
+def test_merge_all_fresh_without_cache(pa, ctx):
+    N, P, D = 700, 4, 128
+    off = W.part_offsets(N, P)
+    of, lf = _gen_states(3, P, 1, 2, N, D, torch.bfloat16)
+    o = torch.empty(1, 2, N, D, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(1, 2, N, device=DEV)
+    pa.pa_merge_states(ctx, off, 1, None, of.to(DEV), lf.to(DEV), None, None, o, lse)
+    ctx.sync_status()
+    ro, rl = O.merge_states(list(of.double().numpy()), list(lf.double().numpy()))
+    assert maxerr(o.float().cpu().numpy(), ro) <= 1e-2
+    assert maxerr(lse.cpu().numpy(), rl) <= 1e-5
+
+
+@pytest.mark.parametrize("N,P,G,B,H", [(1000, 8, 1, 1, 3), (2900, 32, 4, 2, 2), (16, 5, 2, 1, 1)])
+def test_importance_standalone(pa, ctx, N, P, G, B, H):
+    off = W.part_offsets(N, P)
+    empty = [p for p in range(P) if off[p + 1] == off[p]]
+    _, lp = _gen_states(4, P, B, H, N, 8, torch.float32, empty)
+    _, l_all = O.merge_states([np.zeros(lp.shape[1:] + (1,))] * P, list(lp.double().numpy()))
+    lse = torch.from_numpy(l_all.astype(np.float32))
+    w = torch.empty(-(-P // G), P, device=DEV)
+    pa.pa_importance(ctx, off, G, lp.to(DEV), lse.to(DEV), w)
+    ctx.sync_status()
+    rw = O.importance(lp.double().numpy(), lse.double().numpy(), off, G)
+    assert maxerr(w.cpu().numpy(), rw) <= 1e-5
+    np.testing.assert_allclose(w.cpu().numpy().sum(axis=1)[np.diff(O.group_bounds(off, G)) > 0], 1.0,
+                               atol=1e-4)
+
+
+# --------------------------------------------------------------------------- partition attention
+def _check_case(pa, ctx, wl, fresh=None):
+    gpu, ora, sel, off, fresh = run_reuse_case(pa, ctx, wl, fresh)
+    tol = TOL[wl.dtype]
+    errs, untouched = compare_states(gpu, ora, sel, tol)
+    werr = maxerr(gpu["w"], ora["w"])
+    assert untouched, "unselected pairs were written"
+    assert errs["of"] <= tol["o"] and errs["oc"] <= tol["o"] and errs["o"] <= tol["o"], errs
+    assert errs["lf"] <= tol["lse"] and errs["lc"] <= tol["lse"] and errs["lse"] <= tol["lse"], errs
+    assert werr <= tol["w"], werr
+    return errs, werr
+
+
+def test_config0_fp32_full_recompute(pa, ctx):
+    _check_case(pa, ctx, W.workload(0))
+
+
+SMALL_BF16 = [
+    dict(grid=(1, 20, 23), H=2, P=4, G=1),             # N=460: ragged partitions and tiles
+    dict(grid=(1, 25, 40), H=2, P=7, G=2, mask="all"),  # N=1000, S=143
+    dict(grid=(1, 10, 30), H=1, P=1, G=1, mask="all"),  # single partition
+    dict(grid=(1, 10, 10), H=2, P=2, G=1),             # N=100 < one tile
+    dict(grid=(2, 16, 16), H=2, P=4, G=1, D=64),       # D = 64
+    dict(grid=(1, 16, 32), H=2, P=4, G=1, B=2),        # batch 2
+    dict(grid=(1, 4, 4), H=1, P=5, G=1, mask="all"),   # N=16, S=4: partition 4 is empty
+]
+
+
+@pytest.mark.parametrize("kw", SMALL_BF16)
+def test_bf16_small_cases(pa, ctx, kw):
+    kw = dict(kw)
+    wl = W.small_variant(W.workload(1), **kw)
+    _check_case(pa, ctx, wl)
+
+
+def test_fp32_small_ragged_case(pa, ctx):
+    wl = W.small_variant(W.workload(0), grid=(1, 13, 23), H=2, P=3, G=1, cache_sigma=0.05,
+                         mask="neighbours", D=128)
+    _check_case(pa, ctx, wl)
+
+
+def test_config1_image_dit_with_reuse(pa, ctx):
+    errs, werr = _check_case(pa, ctx, W.workload(1))
+    print("config 1", errs, werr)
+
+
+def test_720p_recipe_reduced_grid(pa, ctx):
+    # the 720p workload's recipe (P=32, G=4, nearest-25% groups, sigma 0.03) on a 3-frame grid
+    wl = W.small_variant(W.workload(2), grid=(3, 45, 80), H=2)
+    assert wl.N == 10800 and wl.N % wl.P != 0
+    errs, werr = _check_case(pa, ctx, wl)
+    print("720p recipe, reduced", errs, werr)
+
+
+# --------------------------------------------------------------------------- validation
+def test_validation_errors(pa, ctx):
+    q = torch.zeros(1, 1, 256, 128, dtype=torch.bfloat16, device=DEV)
+    o = torch.zeros(2, 1, 1, 256, 128, dtype=torch.bfloat16, device=DEV)
+    l = torch.zeros(2, 1, 1, 256, device=DEV)
+    off = [0, 128, 256]
+    with pytest.raises(pa.PAError, match="PA_EINVAL"):
+        pa.pa_partition_attn(ctx, q, q, q, [0, 100, 200], 1, None, o, l)     # part_off[P] != N
+    with pytest.raises(pa.PAError, match="PA_EINVAL"):
+        pa.pa_partition_attn(ctx, q, q, q, [0, 200, 100, 256], 1, None, o, l)  # decreasing
+    with pytest.raises(pa.PAError, match="PA_EINVAL"):
+        pa.pa_partition_attn(ctx, q, q, q, off, 3, None, o, l)                 # G > P
+    with pytest.raises(pa.PAError, match="PA_EUNSUPPORTED"):
+        q96 = torch.zeros(1, 1, 256, 96, dtype=torch.bfloat16, device=DEV)
+        pa.pa_partition_attn(ctx, q96, q96, q96, off, 1, None, o, l)
+    with pytest.raises(pa.PAError, match="PA_EUNSUPPORTED"):
+        qh = torch.zeros(1, 1, 256, 128, dtype=torch.float16, device=DEV)
+        pa.pa_partition_attn(ctx, qh, qh, qh, off, 1, None, o, l)
+    flat = torch.zeros(256 * 128 + 8, dtype=torch.bfloat16, device=DEV)
+    mis = flat[1:1 + 256 * 128].view(1, 1, 256, 128)                        # 2-byte offset
+    with pytest.raises(pa.PAError, match="PA_EALIGN"):
+        pa.pa_partition_attn(ctx, mis, q, q, off, 1, None, o, l)
+    ob = torch.zeros(1, 1, 256, 128, dtype=torch.bfloat16, device=DEV)
+    lb = torch.zeros(1, 1, 256, device=DEV)
+    with pytest.raises(pa.PAError, match="PA_EINVAL"):                      # reuse without a cache
+        pa.pa_merge_states(ctx, off, 1, np.array([[1, 0], [0, 1]]), o, l, None, None, ob, lb)
+    with pytest.raises(pa.PAError, match="PA_EINVAL"):
+        pa.pa_relayout_seq2head(ctx, q[0, 0].view(256, 1, 128), q[0, 0].view(1, 256, 128), 4, 4)
+    ctx.sync_status()
+
+
+def test_empty_sequence_is_a_no_op(pa, ctx):
+    q = torch.zeros(1, 1, 0, 128, dtype=torch.bfloat16, device=DEV)
+    o = torch.zeros(1, 1, 1, 0, 128, dtype=torch.bfloat16, device=DEV)
+    l = torch.zeros(1, 1, 1, 0, device=DEV)
+    pa.pa_partition_attn(ctx, q, q, q, [0, 0], 1, None, o, l)
+    ctx.sync_status()
