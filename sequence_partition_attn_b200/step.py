@@ -1,0 +1,166 @@
+"""Device-resident attention step with selective state reuse, built on the libpa calls.
+
+A step takes Q, K, V of one denoising step already in HBM, computes the attention states of
+the fresh (query group, KV group) pairs, and merges them with the cached states of the
+other pairs into (O, LSE) plus the partition importance w (DiTango web summary,
+Methodology 1-2).  ``Trajectory`` adds the host side of the selection: all pairs fresh at
+anchor steps (importance stored, cache refreshed), otherwise pairs whose stored
+importance falls below a threshold reuse the anchor's states.
+
+Only orchestration lives here; every arithmetic step runs in libpa's kernels.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import (Context, pa_merge_states, pa_partition_attn, pa_relayout_seq2head,
+               select_fresh)
+
+
+def attn_flops(part_off, G: int, fresh, B: int, H: int, D: int) -> float:
+    """Algorithmic flops of the fresh pairs: 4*D per (query row, valid key) of each pair
+    (QK^T and PV, multiply-add = 2).  Padding, skipped pairs and exponentials excluded."""
+    off = np.asarray(part_off, dtype=np.int64)
+    P = len(off) - 1
+    QG = -(-P // G)
+    gb = np.array([off[min(g * G, P)] for g in range(QG + 1)])
+    rows = np.diff(gb)
+    total = 0
+    for qg in range(QG):
+        for kg in range(QG):
+            if fresh is None or fresh[qg][kg]:
+                total += int(rows[qg]) * int(rows[kg])
+    return 4.0 * D * B * H * total
+
+
+def merge_bytes(B, H, N, D, P, elem_bytes, with_w=True) -> float:
+    """Algorithmic HBM bytes of the merge: per row P states of (D*elem + 4) read and one
+    state written; the importance adds nothing (fused)."""
+    row = D * elem_bytes + 4
+    return float(B) * H * N * (P * row + row)
+
+
+class AttentionStep:
+    """Buffers and launches of one attention step at a fixed shape, partitioning and mask."""
+
+    def __init__(self, ctx: Context, B, H, N, D, part_off, G, fresh, dtype=torch.bfloat16,
+                 device="cuda:0"):
+        self.ctx = ctx
+        self.B, self.H, self.N, self.D, self.G = B, H, N, D, G
+        self.part_off = np.asarray(part_off, dtype=np.int32)
+        self.P = len(self.part_off) - 1
+        self.QG = -(-self.P // G)
+        self.fresh = None if fresh is None else np.asarray(fresh, dtype=np.uint8)
+        dev = torch.device(device)
+        P = self.P
+        mk = lambda *s, dt=dtype: torch.empty(*s, dtype=dt, device=dev)   # noqa: E731
+        self.q, self.k, self.v = mk(B, H, N, D), mk(B, H, N, D), mk(B, H, N, D)
+        self.o_fresh, self.lse_fresh = mk(P, B, H, N, D), mk(P, B, H, N, dt=torch.float32)
+        reuse = self.fresh is not None and not self.fresh.all()
+        self.o_cached = mk(P, B, H, N, D) if reuse else None
+        self.lse_cached = mk(P, B, H, N, dt=torch.float32) if reuse else None
+        self.o, self.lse = mk(B, H, N, D), mk(B, H, N, dt=torch.float32)
+        self.w = mk(self.QG, P, dt=torch.float32)
+        self.flops = attn_flops(self.part_off, G, self.fresh, B, H, D)
+        self.merge_bytes = merge_bytes(B, H, N, D, P, torch.empty(0, dtype=dtype).element_size())
+
+    def fill_cache(self, k_prev, v_prev, stream=None):
+        """States of every pair on (Q, K_prev, V_prev): the cache of an earlier step."""
+        if self.o_cached is None:
+            return
+        pa_partition_attn(self.ctx, self.q, k_prev, v_prev, self.part_off, self.G, None,
+                          self.o_cached, self.lse_cached, stream=stream)
+
+    def attention(self, stream=None):
+        pa_partition_attn(self.ctx, self.q, self.k, self.v, self.part_off, self.G, self.fresh,
+                          self.o_fresh, self.lse_fresh, stream=stream)
+
+    def merge(self, stream=None):
+        pa_merge_states(self.ctx, self.part_off, self.G, self.fresh, self.o_fresh, self.lse_fresh,
+                        self.o_cached, self.lse_cached, self.o, self.lse, self.w, stream=stream)
+
+    def run(self, stream=None):
+        self.attention(stream)
+        self.merge(stream)
+
+
+class Trajectory:
+    """Denoising trajectory with anchor steps and importance-driven reuse (host selection).
+
+    At an anchor step every pair is fresh, the states become the cache and the importance
+    w is stored (copied to the host: QG*P floats, the only device-to-host transfer).  At
+    any other step the mask is ``select_fresh(w_stored, G, threshold)``; fresh pairs are
+    recomputed from the current K, V and merged with the anchor's cached states.
+    """
+
+    def __init__(self, ctx, B, H, N, D, part_off, G, anchors, threshold, dtype=torch.bfloat16,
+                 device="cuda:0"):
+        self.ctx = ctx
+        self.anchors = set(anchors)
+        self.threshold = threshold
+        self.G = G
+        self.part_off = np.asarray(part_off, dtype=np.int32)
+        P = len(self.part_off) - 1
+        self.P, self.QG = P, -(-P // G)
+        dev = torch.device(device)
+        self.cache_o = torch.empty(P, B, H, N, D, dtype=dtype, device=dev)
+        self.cache_lse = torch.empty(P, B, H, N, dtype=torch.float32, device=dev)
+        self.o_fresh = torch.empty_like(self.cache_o)
+        self.lse_fresh = torch.empty_like(self.cache_lse)
+        self.o = torch.empty(B, H, N, D, dtype=dtype, device=dev)
+        self.lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+        self.w = torch.empty(self.QG, P, dtype=torch.float32, device=dev)
+        self.w_stored = None
+
+    def step(self, s: int, q, k, v, stream=None) -> np.ndarray:
+        """Run step s on device tensors q, k, v; returns the mask it used (uint8[QG, KG])."""
+        if s in self.anchors or self.w_stored is None:
+            mask = np.ones((self.QG, self.QG), dtype=np.uint8)
+            pa_partition_attn(self.ctx, q, k, v, self.part_off, self.G, None, self.cache_o,
+                              self.cache_lse, stream=stream)
+            pa_merge_states(self.ctx, self.part_off, self.G, None, self.cache_o, self.cache_lse,
+                            None, None, self.o, self.lse, self.w, stream=stream)
+            self.w_stored = self.w.cpu().numpy().astype(np.float64)
+            return mask
+        mask = select_fresh(self.w_stored, self.G, self.threshold)
+        pa_partition_attn(self.ctx, q, k, v, self.part_off, self.G, mask, self.o_fresh,
+                          self.lse_fresh, stream=stream)
+        pa_merge_states(self.ctx, self.part_off, self.G, mask, self.o_fresh, self.lse_fresh,
+                        self.cache_o, self.cache_lse, self.o, self.lse, self.w, stream=stream)
+        return mask
+
+
+def relayout_overlapped(ctx, src_qkv, dst_qkv, n_chunks, part_off, G, o_part, lse_part,
+                        s_copy, s_attn):
+    """Chunked seq-major -> head-major relayout of Q, K, V on one stream, overlapped with
+    partition attention over the chunks already moved on another (SwiftFusion web summary,
+    Methodology 2, Torus Attention).  All pairs fresh.
+
+    Chunk c is relayed out (3 launches) and recorded; the attention stream waits for it and
+    computes the new pairs: query chunk c against KV chunks <= c, and query chunks < c
+    against KV chunk c.  Chunk boundaries must be partition boundaries.
+    """
+    src_q, src_k, src_v = src_qkv
+    q, k, v = dst_qkv
+    P = len(part_off) - 1
+    per = P // n_chunks
+    assert per * n_chunks == P and per % G == 0
+    QG = -(-P // G)
+    gpc = per // G                          # groups per chunk
+    events = []
+    for c in range(n_chunks):
+        with torch.cuda.stream(s_copy):
+            for s, d in ((src_q, q), (src_k, k), (src_v, v)):
+                pa_relayout_seq2head(ctx, s, d.view(d.shape[-3], d.shape[-2], d.shape[-1]),
+                                     n_chunks=n_chunks, chunk=c, stream=s_copy)
+            ev = torch.cuda.Event()
+            ev.record(s_copy)
+            events.append(ev)
+        s_attn.wait_event(ev)
+        mask = np.zeros((QG, QG), dtype=np.uint8)
+        lo, hi = c * gpc, (c + 1) * gpc
+        mask[lo:hi, :hi] = 1                # query chunk c x KV chunks <= c
+        mask[:lo, lo:hi] = 1                # query chunks < c x KV chunk c
+        pa_partition_attn(ctx, q, k, v, part_off, G, mask, o_part, lse_part, stream=s_attn)
+    return events

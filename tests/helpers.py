@@ -27,7 +27,8 @@ def maxerr(a, b, mask=None):
     if mask is not None:
         a, b = a[mask], b[mask]
     both_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
-    d = np.where(both_inf, 0.0, np.abs(a - b))
+    with np.errstate(invalid="ignore"):
+        d = np.where(both_inf, 0.0, np.abs(a - b))
     if d.size and np.isnan(d).any():
         return float("inf")                 # a NaN where a value is due fails every tolerance
     return float(d.max()) if d.size else 0.0

@@ -100,8 +100,8 @@ def test_merge_with_reuse_and_fused_importance(pa, ctx, dt, D, N, P, G, B, H):
     ro, rl, ch = O.merge_with_reuse(f64(of), f64(lf), f64(oc), f64(lc), off, G, fresh)
     rw = O.importance(ch, rl, off, G)
     tol = TOL["bf16" if dt == torch.bfloat16 else "f32"]
-    # stored states are exact inputs; only the merge arithmetic and output rounding differ
-    o_tol = 1e-2 if dt == torch.bfloat16 else 1e-5
+    # stored states are exact inputs; the merge arithmetic is fp32 and O is rounded to dtype
+    o_tol = tol["o"] if dt == torch.bfloat16 else 1e-5
     assert maxerr(o.float().cpu().numpy(), ro) <= o_tol
     assert maxerr(lse.cpu().numpy(), rl) <= 1e-5 + 1e-6 * np.abs(rl).max()
     assert maxerr(w.cpu().numpy(), rw) <= tol["w"]
@@ -116,7 +116,7 @@ def test_merge_all_fresh_without_cache(pa, ctx):
     pa.pa_merge_states(ctx, off, 1, None, of.to(DEV), lf.to(DEV), None, None, o, lse)
     ctx.sync_status()
     ro, rl = O.merge_states(list(of.double().numpy()), list(lf.double().numpy()))
-    assert maxerr(o.float().cpu().numpy(), ro) <= 1e-2
+    assert maxerr(o.float().cpu().numpy(), ro) <= TOL["bf16"]["o"]
     assert maxerr(lse.cpu().numpy(), rl) <= 1e-5
 
 
