@@ -6,20 +6,37 @@
 // This is the per-partition state of the DiTango web summary (Methodology 2, "State
 // Composition"; the ring-based group state computation iterates partitions the same way).
 //
-// One CTA owns one 128-row query tile of one (batch, head) and walks every fresh KV
-// partition of its query group in order.  The running softmax restarts at each partition
-// boundary, where the epilogue writes (O_p, LSE_p).
+// One CTA owns two 128-row query tiles (a, b) of one (batch, head) and query group and
+// walks every fresh KV partition of the group in order; each K/V tile is loaded once for
+// both query tiles.  The running softmax restarts at each partition boundary, where the
+// epilogue writes (O_p, LSE_p).
 //
-// Roles (192 threads):
-//   warp 0      TMA producer: Q once, then K and V tiles of 128 keys into a 2-stage ring.
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T into TMEM, then O += P V into TMEM.
-//   warps 2..5  softmax warpgroup, one query row per thread (TMEM lane = row): reads S
-//               from TMEM, masks keys past the partition end, keeps the running max and
-//               sum in the log2 domain, rescales O in TMEM when the max grows, writes
-//               P (bf16) to shared memory for the PV product, and runs the epilogue.
+// Roles (384 threads = 3 warpgroups, one CTA per SM, all 512 TMEM columns).  Launched at
+// 168 registers per thread; warpgroup 0 drops to 56 and the two softmax warpgroups rise to
+// 224 (56 + 2 * 224 = 3 * 168: the split uses exactly the launch allocation).
+//   warp 0      TMA producer: Q_a and Q_b once, then K and V tiles of 128 keys into a
+//               2-stage ring.
+//   warp 1      TMEM owner and MMA issuer.  Order per KV tile j:
+//                 PV_a(j), S_a(j+1), PV_b(j), S_b(j+1)
+//               so that while one softmax warpgroup works on its scores the tensor pipe
+//               runs the other tile's products (ping-pong).
+//   warps 2, 3  idle.
+//   warps 4..7  softmax of tile a; warps 8..11 softmax of tile b.  One query row per
+//               thread (TMEM lane = row).  S (fp32) is read from TMEM, keys past the
+//               partition end are masked, the running max is kept in the log2 domain and
+//               only moved (with a rescale of O in TMEM) when it grows by more than 8
+//               (2^8 bounds P), P is rounded to bf16 and written back over S in TMEM, and
+//               the PV product reads it from there (A operand in TMEM).
 //
-// Overlap: the MMA warp issues S(j+1) as soon as the softmax has released S(j), so the
-// exponentials of tile j+1 run while PV(j) occupies the tensor pipe.
+// Ordering facts the pipeline relies on: tcgen05.mma from one thread executes in issue
+// order and tcgen05.commit tracks every earlier MMA of the thread.  So the completion of
+// S_x(j+1) implies PV_x(j) is complete: the softmax may overwrite S_x / P_x columns and
+// touch O_x after waiting only for S_x(j+1).
+//
+// Exponentials: 2^t on full tiles is split between the MUFU unit (3/4 of the columns) and
+// a degree-3 polynomial on the FMA pipe (1/4): Cody-Waite split t = n + f, |f| <= 1/2,
+// 2^f by a minimax polynomial fitted for this kernel (fit_exp2_poly.py, max relative
+// error 7.5e-5), 2^n added to the exponent field.
 #include "pa_device.cuh"
 #include "pa_launch.h"
 
@@ -29,36 +46,66 @@ namespace {
 constexpr int kBM = 128;        // query rows per tile (MMA M)
 constexpr int kBN = 128;        // keys per tile (MMA N of S, K of PV)
 constexpr int kStages = 2;      // K/V ring depth
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
+constexpr int kRegsLow = 56;      // warpgroup 0 (producer, MMA issuer)
+constexpr int kRegsHigh = 224;    // softmax warpgroups
+static_assert(kRegsLow + 2 * kRegsHigh == 3 * 168, "register split must equal the launch allocation");
 constexpr int kAtomBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16): one swizzle-128B box
 
 template <int D>
 struct Layout {
   static constexpr int kAtoms = D / 64;
   static constexpr int kTileBytes = kAtoms * kAtomBytes;   // a 128 x D bf16 tile
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kQ = 0;                             // Q_a, Q_b
+  static constexpr int kK = kQ + 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kP = kV + kStages * kTileBytes;
-  static constexpr int kBar = kP + 2 * kAtomBytes;         // P: 128 rows x 128 keys bf16
+  static constexpr int kBar = kV + kStages * kTileBytes;
   enum { Q_FULL = 0, K_FULL = 1, V_FULL = K_FULL + kStages, KV_EMPTY = V_FULL + kStages,
-         S_FULL = KV_EMPTY + kStages, P_FULL, O_DONE, NBAR };
+         S_FULL = KV_EMPTY + kStages, P_FULL = S_FULL + 2, O_DONE = P_FULL + 2, NBAR = O_DONE + 2 };
   static constexpr int kTmemSlot = kBar + NBAR * 8;
   static constexpr int kAbort = kTmemSlot + 8;
   static constexpr int kUsed = kAbort + 8;
   static constexpr int kSmemBytes = kUsed + 1024;          // slack for 1024-byte alignment
-  static constexpr uint32_t kTmemCols = 256;               // S: 128 columns, O: D columns
+  static constexpr uint32_t kTmemCols = 512;               // S_a, S_b, O_a, O_b: 128 each
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  static_assert(128 + D <= (int)kTmemCols, "TMEM budget");
 };
 
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleLog2 = 8.0f;    // move the running max only when it grows by > 8
+
+// Minimax coefficients of 2^f on [-1/2, 1/2] (relative error), from fit_exp2_poly.py.
+constexpr float kC0 = 0.9999280571937561f;
+constexpr float kC1 = 0.6932609677314758f;
+constexpr float kC2 = 0.24261093139648438f;
+constexpr float kC3 = 0.05517149344086647f;
+
+// 2^t on the FMA pipe.  t is clamped at -126 so that adding n to the exponent field of
+// 2^f (which lies in [0.70, 1.42]) can never underflow the field.
+__device__ __forceinline__ float poly_exp2(float t) {
+  t = fmaxf(t, -126.0f);
+  const float rnd = t + 12582912.0f;          // 1.5 * 2^23: n = round(t) lands in the low bits
+  const float n = rnd - 12582912.0f;
+  const float f = t - n;
+  const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(rnd) << 23));
+}
 
 // Next partition >= from that is fresh for query group qg and holds at least one key.
 __device__ __forceinline__ int next_part(const AttnTables& t, int qg, int from) {
   for (int p = from; p < t.P; ++p)
     if (fresh_bit(t.fresh_bits, qg, p) && t.part_off[p + 1] > t.part_off[p]) return p;
   return t.P;
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16; A (M x 16) is read from TMEM columns.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 template <int D>
@@ -76,16 +123,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Decode the work unit: (b*H + h, query group, 128-row tile of the group).
+  // Decode the work unit: (b*H + h, query group, 256-row block of the group).
   const int bh = blockIdx.x / prm.tiles_total;
   const int tix = blockIdx.x - bh * prm.tiles_total;
   int qg = 0;
   while (qg + 1 < t.QG && t.tile_start[qg + 1] <= tix) ++qg;
-  const int q_row0 = t.qg_row0[qg] + (tix - t.tile_start[qg]) * kBM;
+  const int q_row0 = t.qg_row0[qg] + (tix - t.tile_start[qg]) * (2 * kBM);
   const int q_end = t.qg_row0[qg + 1];
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < L::NBAR; ++i) mbar_init(bar(i), i == L::P_FULL ? 128u : 1u);
+    for (int i = 0; i < L::NBAR; ++i)
+      mbar_init(bar(i), (i == L::P_FULL || i == L::P_FULL + 1) ? 128u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -97,23 +145,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(gbase + L::kTmemSlot);
-  const uint32_t tS = tmem;          // columns [0, 128)
-  const uint32_t tO = tmem + 128;    // columns [128, 128 + D)
 
   const uint32_t sQ = base + L::kQ;
-  const uint32_t sP = base + L::kP;
   auto sK = [&](int s) { return base + L::kK + (uint32_t)s * L::kTileBytes; };
   auto sV = [&](int s) { return base + L::kV + (uint32_t)s * L::kTileBytes; };
 
+  if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       tma_prefetch(&prm.tm_q);
       tma_prefetch(&prm.tm_k);
       tma_prefetch(&prm.tm_v);
-      mbar_expect_tx(bar(L::Q_FULL), L::kTileBytes);
-      for (int a = 0; a < L::kAtoms; ++a)
-        tma_load_3d(sQ + a * kAtomBytes, &prm.tm_q, a * 64, q_row0, bh, bar(L::Q_FULL));
+      mbar_expect_tx(bar(L::Q_FULL), 2 * L::kTileBytes);
+      for (int x = 0; x < 2; ++x)
+        for (int a = 0; a < L::kAtoms; ++a)
+          tma_load_3d(sQ + x * L::kTileBytes + a * kAtomBytes, &prm.tm_q, a * 64, q_row0 + x * kBM, bh,
+                      bar(L::Q_FULL));
       int j = 0;
       bool ok = true;
       for (int p = next_part(t, qg, 0); ok && p < t.P; p = next_part(t, qg, p + 1)) {
@@ -144,17 +192,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16(kBM, kBN, false, false);   // Q K-major, K K-major
-      constexpr uint32_t kIdPV = idesc_bf16(kBM, D, false, true);     // P K-major, V MN-major
+      constexpr uint32_t kIdPV = idesc_bf16(kBM, D, false, true);     // P (TMEM), V MN-major
       int T = 0;
       for (int p = next_part(t, qg, 0); p < t.P; p = next_part(t, qg, p + 1))
         T += (t.part_off[p + 1] - t.part_off[p] + kBN - 1) / kBN;
-      auto issue_s = [&](int s) {
+      auto issue_s = [&](int x, int s) {
+        const uint32_t q = sQ + x * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
-          mma_bf16_ss(tS, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK(s) + off, 16, 1024),
-                      kIdS, kk > 0);
+          mma_bf16_ss(tmem + x * 128, smem_desc_sw128(q + off, 16, 1024),
+                      smem_desc_sw128(sK(s) + off, 16, 1024), kIdS, kk > 0);
         }
+        mma_commit(bar(L::S_FULL + x));
+      };
+      auto issue_pv = [&](int x, int s, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_bf16_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
+                      smem_desc_sw128(sV(s) + kk * 16 * 128, kAtomBytes, 1024), kIdPV,
+                      (first && kk == 0) ? 0u : 1u);
+        mma_commit(bar(L::O_DONE + x));
       };
       bool ok = mbar_wait(bar(L::Q_FULL), 0, abort_flag, status);
       int j = 0;
@@ -162,40 +220,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         ok = mbar_wait(bar(L::K_FULL + 0), 0, abort_flag, status);
         if (ok) {
           tc_fence_after();
-          issue_s(0);
-          mma_commit(bar(L::S_FULL));
+          issue_s(0, 0);
+          issue_s(1, 0);
         }
         int p = next_part(t, qg, 0);
         int key = t.part_off[p];
         for (; ok && j < T; ++j) {
           const bool first = key == t.part_off[p];
-          if (!mbar_wait(bar(L::P_FULL), j & 1, abort_flag, status)) { ok = false; break; }
+          const int s = j % kStages, s1 = (j + 1) % kStages;
+          const bool more = j + 1 < T;
+          if (!mbar_wait(bar(L::P_FULL + 0), j & 1, abort_flag, status)) { ok = false; break; }
+          if (!mbar_wait(bar(L::V_FULL + s), (j / kStages) & 1, abort_flag, status)) { ok = false; break; }
           tc_fence_after();
-          if (j + 1 < T) {
-            const int s1 = (j + 1) % kStages;
+          issue_pv(0, s, first);
+          if (more) {
             if (!mbar_wait(bar(L::K_FULL + s1), ((j + 1) / kStages) & 1, abort_flag, status)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            issue_s(s1);
-            mma_commit(bar(L::S_FULL));
+            issue_s(0, s1);
           }
-          const int s = j % kStages;
-          if (!mbar_wait(bar(L::V_FULL + s), (j / kStages) & 1, abort_flag, status)) {
-            ok = false;
-            break;
-          }
+          if (!mbar_wait(bar(L::P_FULL + 1), j & 1, abort_flag, status)) { ok = false; break; }
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint32_t aoff = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
-            mma_bf16_ss(tO, smem_desc_sw128(sP + aoff, 16, 1024),
-                        smem_desc_sw128(sV(s) + kk * 16 * 128, kAtomBytes, 1024), kIdPV,
-                        (first && kk == 0) ? 0u : 1u);
-          }
-          mma_commit(bar(L::O_DONE));
+          issue_pv(1, s, first);
           mma_commit(bar(L::KV_EMPTY + s));
+          if (more) issue_s(1, s1);
           key += kBN;
           if (key >= t.part_off[p + 1]) {
             p = next_part(t, qg, p + 1);
@@ -207,13 +257,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       for (int jj = (j > kStages ? j - kStages : 0); jj < j; ++jj)
         mbar_drain(bar(L::KV_EMPTY + jj % kStages), (jj / kStages) & 1);
     }
-  } else {
-    // ---------------------------------------------------------------- softmax warpgroup
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- softmax warpgroups
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+    const int x = (warp - 4) >> 2;                 // query tile: 0 = a (warps 4-7), 1 = b
     const int wq = warp & 3;                       // TMEM lane quarter this warp may access
     const int row = wq * 32 + lane;
-    const int q_row = q_row0 + row;
+    const int q_row = q_row0 + x * kBM + row;
     const bool row_ok = q_row < q_end;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + x * 128;
+    const uint32_t tO = tmem + lane_off + 256 + x * 128;
     const size_t BHN = static_cast<size_t>(prm.BH) * prm.N;
     __nv_bfloat16* o_part = static_cast<__nv_bfloat16*>(prm.o_part);
 
@@ -233,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(tO + lane_off + c * 32, v);
+        tmem_ld32(tO + c * 32, v);
         tmem_wait_ld();
         if (row_ok) {
 #pragma unroll
@@ -250,92 +304,94 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if (row_ok) prm.lse_part[r] = (m + fast_log2(l)) * kLn2;
     };
 
-    float m = -INFINITY, l = 0.0f;
+    float m = -INFINITY, l = 0.0f;   // running max (log2 units, scaled) and sum
     int j = 0, prev = -1;
     bool ok = true;
     const float sl2 = prm.scale_log2;
     for (int p = next_part(t, qg, 0); ok && p < t.P; p = next_part(t, qg, p + 1)) {
       const int k0 = t.part_off[p], k1 = t.part_off[p + 1];
       for (int key = k0; key < k1; key += kBN, ++j) {
-        if (!mbar_wait(bar(L::S_FULL), j & 1, abort_flag, status)) { ok = false; break; }
+        if (!mbar_wait(bar(L::S_FULL + x), j & 1, abort_flag, status)) { ok = false; break; }
         tc_fence_after();
-        float x[kBN];
+        float s[kBN];
         {
           uint32_t r0[32], r1[32], r2[32], r3[32];
-          tmem_ld32(tS + lane_off + 0, r0);
-          tmem_ld32(tS + lane_off + 32, r1);
-          tmem_ld32(tS + lane_off + 64, r2);
-          tmem_ld32(tS + lane_off + 96, r3);
+          tmem_ld32(tS + 0, r0);
+          tmem_ld32(tS + 32, r1);
+          tmem_ld32(tS + 64, r2);
+          tmem_ld32(tS + 96, r3);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            x[i] = __uint_as_float(r0[i]);
-            x[32 + i] = __uint_as_float(r1[i]);
-            x[64 + i] = __uint_as_float(r2[i]);
-            x[96 + i] = __uint_as_float(r3[i]);
+            s[i] = __uint_as_float(r0[i]);
+            s[32 + i] = __uint_as_float(r1[i]);
+            s[64 + i] = __uint_as_float(r2[i]);
+            s[96 + i] = __uint_as_float(r3[i]);
           }
         }
         const int nvalid = min(kBN, k1 - key);
-        float mt = -INFINITY;
+        if (nvalid < kBN) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          x[c] = c < nvalid ? x[c] * sl2 : -INFINITY;
-          mt = fmaxf(mt, x[c]);
+          for (int c = 0; c < kBN; ++c) s[c] = c < nvalid ? s[c] : -INFINITY;
         }
-        // PV(j-1) must be complete before O is rescaled or read and before P is rewritten.
-        if (j > 0) {
-          if (!mbar_wait(bar(L::O_DONE), (j - 1) & 1, abort_flag, status)) { ok = false; break; }
-          tc_fence_after();
-        }
+        float mt = s[0];
+#pragma unroll
+        for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, s[c]);
+        mt *= sl2;
         if (key == k0) {
+          // S_x(j) complete implies PV_x(j-1) complete: O_x holds the previous partition.
           if (prev >= 0) epilogue(prev, m, l);
           m = mt;
           l = 0.0f;
-        } else {
+        } else if (__any_sync(0xffffffffu, mt - m > kRescaleLog2)) {
           const float m_new = fmaxf(m, mt);
           const float alpha = fast_exp2(m - m_new);
-          if (__any_sync(0xffffffffu, m_new > m)) {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t v[32];
-              tmem_ld32(tO + lane_off + c * 32, v);
-              tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tO + c * 32, v);
+            tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-              tmem_st32(tO + lane_off + c * 32, v);
-            }
-            tmem_wait_st();
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+            tmem_st32(tO + c * 32, v);
           }
           l *= alpha;
           m = m_new;
         }
         float rs = 0.0f;
+        if (nvalid == kBN) {
 #pragma unroll
-        for (int c = 0; c < kBN; ++c) {
-          x[c] = fast_exp2(x[c] - m);
-          rs += x[c];
+          for (int c = 0; c < kBN; ++c) {
+            const float a = fmaf(s[c], sl2, -m);
+            s[c] = (c & 7) >= 6 ? poly_exp2(a) : fast_exp2(a);
+            rs += s[c];
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kBN; ++c) {
+            s[c] = fast_exp2(fmaf(s[c], sl2, -m));     // exp2(-inf) = 0 for masked keys
+            rs += s[c];
+          }
         }
         l += rs;
-        // P row -> shared memory, K-major with the 128-byte swizzle (16-byte chunk index
-        // XOR row % 8 inside each 1024-byte group of 8 rows).
+        // P (bf16, two per 32-bit column) over the first 64 columns of S_x.
+        {
+          uint32_t w0[32], w1[32];
 #pragma unroll
-        for (int ch = 0; ch < kBN / 8; ++ch) {
-          const uint32_t addr = sP + (ch >> 3) * kAtomBytes + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-          const uint32_t w0 = pack_bf16x2(x[ch * 8 + 0], x[ch * 8 + 1]);
-          const uint32_t w1 = pack_bf16x2(x[ch * 8 + 2], x[ch * 8 + 3]);
-          const uint32_t w2 = pack_bf16x2(x[ch * 8 + 4], x[ch * 8 + 5]);
-          const uint32_t w3 = pack_bf16x2(x[ch * 8 + 6], x[ch * 8 + 7]);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
-                       "r"(w2), "r"(w3)
-                       : "memory");
+          for (int i = 0; i < 32; ++i) {
+            w0[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
+            w1[i] = pack_bf16x2(s[64 + 2 * i], s[64 + 2 * i + 1]);
+          }
+          tmem_st32(tS + 0, w0);
+          tmem_st32(tS + 32, w1);
         }
-        fence_async_smem();
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(L::P_FULL));
+        mbar_arrive(bar(L::P_FULL + x));
         prev = p;
       }
     }
-    if (ok && j > 0 && mbar_wait(bar(L::O_DONE), (j - 1) & 1, abort_flag, status)) {
+    if (ok && j > 0 && mbar_wait(bar(L::O_DONE + x), (j - 1) & 1, abort_flag, status)) {
       tc_fence_after();
       epilogue(prev, m, l);
     }
@@ -364,6 +420,7 @@ int launch_attn_tc(const TcParams& prm, int units, cudaStream_t st) {
   return prm.D == 64 ? launch_impl<64>(prm, units, st) : launch_impl<128>(prm, units, st);
 }
 
-int attn_tc_tile_rows() { return kBM; }
+// Query rows per work unit (two 128-row tiles).
+int attn_tc_tile_rows() { return 2 * kBM; }
 
 }  // namespace pa
