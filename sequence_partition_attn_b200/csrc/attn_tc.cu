@@ -33,10 +33,10 @@
 // S_x(j+1) implies PV_x(j) is complete: the softmax may overwrite S_x / P_x columns and
 // touch O_x after waiting only for S_x(j+1).
 //
-// Exponentials: 2^t on full tiles is split between the MUFU unit (3/4 of the columns) and
-// a degree-3 polynomial on the FMA pipe (1/4): Cody-Waite split t = n + f, |f| <= 1/2,
-// 2^f by a minimax polynomial fitted for this kernel (fit_exp2_poly.py, max relative
-// error 7.5e-5), 2^n added to the exponent field.
+// Exponentials: 2^t on full tiles can be split between the MUFU unit and a degree-3
+// polynomial on the FMA pipe (kPolyCols of every 8 columns): Cody-Waite split t = n + f,
+// |f| <= 1/2, 2^f by a minimax polynomial fitted for this kernel (fit_exp2_poly.py, max
+// relative error 7.5e-5), 2^n added to the exponent field.
 #include "pa_device.cuh"
 #include "pa_launch.h"
 
@@ -72,6 +72,11 @@ struct Layout {
 
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;    // move the running max only when it grows by > 8
+// Columns out of every 8 whose exponential runs on the FMA pipe (polynomial) instead of
+// MUFU.  Measured on B200 at the 720p shape: 0 -> 893, 1 -> 891, 2 -> 859, 3 -> 817,
+// 4 -> 779 TFLOP/s, so the MUFU unit is not the limiter of this kernel and all
+// exponentials go to it.
+constexpr int kPolyCols = 0;
 
 // Minimax coefficients of 2^f on [-1/2, 1/2] (relative error), from fit_exp2_poly.py.
 constexpr float kC0 = 0.9999280571937561f;
@@ -88,6 +93,26 @@ __device__ __forceinline__ float poly_exp2(float t) {
   const float f = t - n;
   const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
   return __int_as_float(__float_as_int(p) + (__float_as_int(rnd) << 23));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Row max of 128 scores: 8 independent 3-input max chains, then a short tree.
+__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = fmax3(s[i], s[i + 8], s[i + 16]);
+#pragma unroll
+  for (int c = 24; c < 120; c += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[120 + i]);
+  return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
 }
 
 // Next partition >= from that is fresh for query group qg and holds at least one key.
@@ -334,10 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
           for (int c = 0; c < kBN; ++c) s[c] = c < nvalid ? s[c] : -INFINITY;
         }
-        float mt = s[0];
-#pragma unroll
-        for (int c = 1; c < kBN; ++c) mt = fmaxf(mt, s[c]);
-        mt *= sl2;
+        const float mt = row_max128(s) * sl2;
         if (key == k0) {
           // S_x(j) complete implies PV_x(j-1) complete: O_x holds the previous partition.
           if (prev >= 0) epilogue(prev, m, l);
@@ -358,22 +380,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           l *= alpha;
           m = m_new;
         }
-        float rs = 0.0f;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 independent sum chains
         if (nvalid == kBN) {
 #pragma unroll
           for (int c = 0; c < kBN; ++c) {
             const float a = fmaf(s[c], sl2, -m);
-            s[c] = (c & 7) >= 6 ? poly_exp2(a) : fast_exp2(a);
-            rs += s[c];
+            s[c] = (c & 7) >= 8 - kPolyCols ? poly_exp2(a) : fast_exp2(a);
+            acc[c & 7] += s[c];
           }
         } else {
 #pragma unroll
           for (int c = 0; c < kBN; ++c) {
             s[c] = fast_exp2(fmaf(s[c], sl2, -m));     // exp2(-inf) = 0 for masked keys
-            rs += s[c];
+            acc[c & 7] += s[c];
           }
         }
-        l += rs;
+        l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         // P (bf16, two per 32-bit column) over the first 64 columns of S_x.
         {
           uint32_t w0[32], w1[32];
