@@ -12,8 +12,8 @@
 // epilogue writes (O_p, LSE_p).
 //
 // Roles (384 threads = 3 warpgroups, one CTA per SM, all 512 TMEM columns).  Launched at
-// 168 registers per thread; warpgroup 0 drops to 56 and the two softmax warpgroups rise to
-// 224 (56 + 2 * 224 = 3 * 168: the split uses exactly the launch allocation).
+// 168 registers per thread; warpgroup 0 drops to 88 and the two softmax warpgroups rise to
+// 208 (88 + 2 * 208 = 3 * 168: the split uses exactly the launch allocation).
 //   warp 0      TMA producer: Q_a and Q_b once, then K and V tiles of 128 keys into a
 //               2-stage ring.
 //   warp 1      TMEM owner and MMA issuer.  Order per KV tile j:
@@ -47,8 +47,8 @@ constexpr int kBM = 128;        // query rows per tile (MMA M)
 constexpr int kBN = 128;        // keys per tile (MMA N of S, K of PV)
 constexpr int kStages = 2;      // K/V ring depth
 constexpr int kThreads = 384;
-constexpr int kRegsLow = 56;      // warpgroup 0 (producer, MMA issuer)
-constexpr int kRegsHigh = 224;    // softmax warpgroups
+constexpr int kRegsLow = 88;      // warpgroup 0 (producer, MMA issuer)
+constexpr int kRegsHigh = 208;    // softmax warpgroups
 static_assert(kRegsLow + 2 * kRegsHigh == 3 * 168, "register split must equal the launch allocation");
 constexpr int kAtomBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16): one swizzle-128B box
 
@@ -131,6 +131,28 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// S_x = Q_x K^T: D/16 MMAs of 128 x 128 x 16 (K-major operands, 128-byte swizzle; the
+// k-step moves 32 bytes inside a 64-element swizzle atom, then to the next atom).
+template <int D>
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t dq, uint64_t dk, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = static_cast<uint32_t>(((kk >> 2) * kAtomBytes + (kk & 3) * 32) >> 4);
+    mma_bf16_ss(d_tmem, dq + off, dk + off, idesc, kk > 0);
+  }
+}
+
+// O_x (+)= P_x V: 8 MMAs of 128 x D x 16; P from TMEM (8 columns = 16 bf16 per k-step), V
+// MN-major (a k-step of 16 keys moves 16 rows of 128 bytes).
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t dv, uint32_t idesc,
+                                         bool first) {
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk)
+    mma_bf16_ts(d_tmem, p_tmem + kk * 8, dv + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc,
+                (first && kk == 0) ? 0u : 1u);
 }
 
 template <int D>
@@ -221,32 +243,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       int T = 0;
       for (int p = next_part(t, qg, 0); p < t.P; p = next_part(t, qg, p + 1))
         T += (t.part_off[p + 1] - t.part_off[p] + kBN - 1) / kBN;
-      auto issue_s = [&](int x, int s) {
-        const uint32_t q = sQ + x * L::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
-          mma_bf16_ss(tmem + x * 128, smem_desc_sw128(q + off, 16, 1024),
-                      smem_desc_sw128(sK(s) + off, 16, 1024), kIdS, kk > 0);
-        }
-        mma_commit(bar(L::S_FULL + x));
-      };
-      auto issue_pv = [&](int x, int s, bool first) {
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_bf16_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
-                      smem_desc_sw128(sV(s) + kk * 16 * 128, kAtomBytes, 1024), kIdPV,
-                      (first && kk == 0) ? 0u : 1u);
-        mma_commit(bar(L::O_DONE + x));
-      };
+      // Descriptors of every operand tile, built once; a k-step only adds to the start
+      // address field (bits 0-13, in 16-byte units).
+      const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dq1 = smem_desc_sw128(sQ + L::kTileBytes, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(sK(0), 16, 1024);
+      const uint64_t dk1 = smem_desc_sw128(sK(1), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(sV(0), kAtomBytes, 1024);
+      const uint64_t dv1 = smem_desc_sw128(sV(1), kAtomBytes, 1024);
       bool ok = mbar_wait(bar(L::Q_FULL), 0, abort_flag, status);
       int j = 0;
       if (ok && T > 0) {
         ok = mbar_wait(bar(L::K_FULL + 0), 0, abort_flag, status);
         if (ok) {
           tc_fence_after();
-          issue_s(0, 0);
-          issue_s(1, 0);
+          issue_s<D>(tmem, dq0, dk0, kIdS);
+          mma_commit(bar(L::S_FULL + 0));
+          issue_s<D>(tmem + 128, dq1, dk0, kIdS);
+          mma_commit(bar(L::S_FULL + 1));
         }
         int p = next_part(t, qg, 0);
         int key = t.part_off[p];
@@ -254,23 +268,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const bool first = key == t.part_off[p];
           const int s = j % kStages, s1 = (j + 1) % kStages;
           const bool more = j + 1 < T;
-          if (!mbar_wait(bar(L::P_FULL + 0), j & 1, abort_flag, status)) { ok = false; break; }
+          const uint64_t dv = s ? dv1 : dv0;
+          const uint64_t dk = s1 ? dk1 : dk0;
+          // Operand waits first (normally already complete), then the softmax hand-offs.
           if (!mbar_wait(bar(L::V_FULL + s), (j / kStages) & 1, abort_flag, status)) { ok = false; break; }
+          if (more && !mbar_wait(bar(L::K_FULL + s1), ((j + 1) / kStages) & 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait(bar(L::P_FULL + 0), j & 1, abort_flag, status)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(0, s, first);
+          issue_pv<D>(tmem + 256, tmem, dv, kIdPV, first);
+          mma_commit(bar(L::O_DONE + 0));
           if (more) {
-            if (!mbar_wait(bar(L::K_FULL + s1), ((j + 1) / kStages) & 1, abort_flag, status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_s(0, s1);
+            issue_s<D>(tmem, dq0, dk, kIdS);
+            mma_commit(bar(L::S_FULL + 0));
           }
           if (!mbar_wait(bar(L::P_FULL + 1), j & 1, abort_flag, status)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(1, s, first);
+          issue_pv<D>(tmem + 384, tmem + 128, dv, kIdPV, first);
+          mma_commit(bar(L::O_DONE + 1));
           mma_commit(bar(L::KV_EMPTY + s));
-          if (more) issue_s(1, s1);
+          if (more) {
+            issue_s<D>(tmem + 128, dq1, dk, kIdS);
+            mma_commit(bar(L::S_FULL + 1));
+          }
           key += kBN;
           if (key >= t.part_off[p + 1]) {
             p = next_part(t, qg, p + 1);
@@ -380,33 +402,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           l *= alpha;
           m = m_new;
         }
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 independent sum chains
+        // Exponentials, row sum (8 independent chains) and P packed to bf16 pairs in one
+        // pass; P goes over the first 64 columns of S_x.
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        uint32_t w[64];
         if (nvalid == kBN) {
 #pragma unroll
-          for (int c = 0; c < kBN; ++c) {
-            const float a = fmaf(s[c], sl2, -m);
-            s[c] = (c & 7) >= 8 - kPolyCols ? poly_exp2(a) : fast_exp2(a);
-            acc[c & 7] += s[c];
+          for (int i = 0; i < 64; ++i) {
+            const int c = 2 * i;
+            const float a0 = fmaf(s[c], sl2, -m), a1 = fmaf(s[c + 1], sl2, -m);
+            const float e0 = (c & 7) >= 8 - kPolyCols ? poly_exp2(a0) : fast_exp2(a0);
+            const float e1 = ((c + 1) & 7) >= 8 - kPolyCols ? poly_exp2(a1) : fast_exp2(a1);
+            acc[c & 7] += e0;
+            acc[(c + 1) & 7] += e1;
+            w[i] = pack_bf16x2(e0, e1);
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < kBN; ++c) {
-            s[c] = fast_exp2(fmaf(s[c], sl2, -m));     // exp2(-inf) = 0 for masked keys
-            acc[c & 7] += s[c];
+          for (int i = 0; i < 64; ++i) {
+            const int c = 2 * i;
+            const float e0 = fast_exp2(fmaf(s[c], sl2, -m));        // exp2(-inf) = 0: masked keys
+            const float e1 = fast_exp2(fmaf(s[c + 1], sl2, -m));
+            acc[c & 7] += e0;
+            acc[(c + 1) & 7] += e1;
+            w[i] = pack_bf16x2(e0, e1);
           }
         }
         l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-        // P (bf16, two per 32-bit column) over the first 64 columns of S_x.
-        {
-          uint32_t w0[32], w1[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            w0[i] = pack_bf16x2(s[2 * i], s[2 * i + 1]);
-            w1[i] = pack_bf16x2(s[64 + 2 * i], s[64 + 2 * i + 1]);
-          }
-          tmem_st32(tS + 0, w0);
-          tmem_st32(tS + 32, w1);
-        }
+        tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&w[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&w[32]));
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(L::P_FULL + x));
