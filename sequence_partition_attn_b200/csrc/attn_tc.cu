@@ -61,7 +61,8 @@ struct Layout {
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kBar = kV + kStages * kTileBytes;
   enum { Q_FULL = 0, K_FULL = 1, V_FULL = K_FULL + kStages, KV_EMPTY = V_FULL + kStages,
-         S_FULL = KV_EMPTY + kStages, P_FULL = S_FULL + 2, O_DONE = P_FULL + 2, NBAR = O_DONE + 2 };
+         S_FULL = KV_EMPTY + kStages, P_LO = S_FULL + 2, P_HI = P_LO + 2, O_DONE = P_HI + 2,
+         NBAR = O_DONE + 2 };
   static constexpr int kTmemSlot = kBar + NBAR * 8;
   static constexpr int kAbort = kTmemSlot + 8;
   static constexpr int kUsed = kAbort + 8;
@@ -77,6 +78,9 @@ constexpr float kRescaleLog2 = 8.0f;    // move the running max only when it gro
 // 4 -> 779 TFLOP/s, so the MUFU unit is not the limiter of this kernel and all
 // exponentials go to it.
 constexpr int kPolyCols = 0;
+// true: the MMA issuer polls the softmax hand-off barriers (test_wait) instead of sleeping
+// on them (try_wait).  Measured at the 720p shape: no difference beyond run-to-run noise.
+constexpr bool kPollHandoff = false;
 
 // Minimax coefficients of 2^f on [-1/2, 1/2] (relative error), from fit_exp2_poly.py.
 constexpr float kC0 = 0.9999280571937561f;
@@ -146,13 +150,32 @@ __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t dq, uint64_t d
 
 // O_x (+)= P_x V: 8 MMAs of 128 x D x 16; P from TMEM (8 columns = 16 bf16 per k-step), V
 // MN-major (a k-step of 16 keys moves 16 rows of 128 bytes).
-template <int D>
+// Half h of the keys: k-steps 4h .. 4h+3.
+template <int D, int H>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t dv, uint32_t idesc,
                                          bool first) {
 #pragma unroll
-  for (int kk = 0; kk < kBN / 16; ++kk)
+  for (int kk = H * 4; kk < H * 4 + 4; ++kk)
     mma_bf16_ts(d_tmem, p_tmem + kk * 8, dv + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc,
                 (first && kk == 0) ? 0u : 1u);
+}
+
+// Exponentials of half H of a row (columns 64H .. 64H+63), added to the 8 row-sum chains
+// and packed to bf16 pairs (32 TMEM columns).  kFull: every key valid (masked keys hold
+// -inf otherwise, and MUFU's exp2(-inf) = 0 handles them).
+template <bool kFull, int H>
+__device__ __forceinline__ void exp_pack_half(const float (&s)[128], float m, float sl2, float (&acc)[8],
+                                              uint32_t (&w)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const int c = H * 64 + 2 * i;
+    const float a0 = fmaf(s[c], sl2, -m), a1 = fmaf(s[c + 1], sl2, -m);
+    const float e0 = (kFull && (c & 7) >= 8 - kPolyCols) ? poly_exp2(a0) : fast_exp2(a0);
+    const float e1 = (kFull && ((c + 1) & 7) >= 8 - kPolyCols) ? poly_exp2(a1) : fast_exp2(a1);
+    acc[c & 7] += e0;
+    acc[(c + 1) & 7] += e1;
+    w[i] = pack_bf16x2(e0, e1);
+  }
 }
 
 template <int D>
@@ -180,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NBAR; ++i)
-      mbar_init(bar(i), (i == L::P_FULL || i == L::P_FULL + 1) ? 128u : 1u);
+      mbar_init(bar(i), (i >= L::P_LO && i < L::O_DONE) ? 128u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -251,6 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint64_t dk1 = smem_desc_sw128(sK(1), 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(sV(0), kAtomBytes, 1024);
       const uint64_t dv1 = smem_desc_sw128(sV(1), kAtomBytes, 1024);
+      auto wait_p = [&](uint32_t b, uint32_t parity) {
+        return kPollHandoff ? mbar_wait_poll(b, parity, abort_flag, status)
+                            : mbar_wait(b, parity, abort_flag, status);
+      };
       bool ok = mbar_wait(bar(L::Q_FULL), 0, abort_flag, status);
       int j = 0;
       if (ok && T > 0) {
@@ -276,17 +303,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             ok = false;
             break;
           }
-          if (!mbar_wait(bar(L::P_FULL + 0), j & 1, abort_flag, status)) { ok = false; break; }
+          if (!wait_p(bar(L::P_LO + 0), j & 1)) { ok = false; break; }
           tc_fence_after();
-          issue_pv<D>(tmem + 256, tmem, dv, kIdPV, first);
+          issue_pv<D, 0>(tmem + 256, tmem, dv, kIdPV, first);
+          if (!wait_p(bar(L::P_HI + 0), j & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv<D, 1>(tmem + 256, tmem, dv, kIdPV, first);
           mma_commit(bar(L::O_DONE + 0));
           if (more) {
             issue_s<D>(tmem, dq0, dk, kIdS);
             mma_commit(bar(L::S_FULL + 0));
           }
-          if (!mbar_wait(bar(L::P_FULL + 1), j & 1, abort_flag, status)) { ok = false; break; }
+          if (!wait_p(bar(L::P_LO + 1), j & 1)) { ok = false; break; }
           tc_fence_after();
-          issue_pv<D>(tmem + 384, tmem + 128, dv, kIdPV, first);
+          issue_pv<D, 0>(tmem + 384, tmem + 128, dv, kIdPV, first);
+          if (!wait_p(bar(L::P_HI + 1), j & 1)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv<D, 1>(tmem + 384, tmem + 128, dv, kIdPV, first);
           mma_commit(bar(L::O_DONE + 1));
           mma_commit(bar(L::KV_EMPTY + s));
           if (more) {
@@ -402,38 +435,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           l *= alpha;
           m = m_new;
         }
-        // Exponentials, row sum (8 independent chains) and P packed to bf16 pairs in one
-        // pass; P goes over the first 64 columns of S_x.
+        // Exponentials, row sum (8 independent chains) and P packed to bf16 pairs, half a
+        // row at a time; each half of P goes over S_x's first 64 columns and is handed to
+        // the MMA issuer at once, so PV on keys 0-63 overlaps the exponentials of 64-127.
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        uint32_t w[64];
-        if (nvalid == kBN) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const int c = 2 * i;
-            const float a0 = fmaf(s[c], sl2, -m), a1 = fmaf(s[c + 1], sl2, -m);
-            const float e0 = (c & 7) >= 8 - kPolyCols ? poly_exp2(a0) : fast_exp2(a0);
-            const float e1 = ((c + 1) & 7) >= 8 - kPolyCols ? poly_exp2(a1) : fast_exp2(a1);
-            acc[c & 7] += e0;
-            acc[(c + 1) & 7] += e1;
-            w[i] = pack_bf16x2(e0, e1);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const int c = 2 * i;
-            const float e0 = fast_exp2(fmaf(s[c], sl2, -m));        // exp2(-inf) = 0: masked keys
-            const float e1 = fast_exp2(fmaf(s[c + 1], sl2, -m));
-            acc[c & 7] += e0;
-            acc[(c + 1) & 7] += e1;
-            w[i] = pack_bf16x2(e0, e1);
-          }
+        {
+          uint32_t w[32];
+          if (nvalid == kBN) exp_pack_half<true, 0>(s, m, sl2, acc, w);
+          else exp_pack_half<false, 0>(s, m, sl2, acc, w);
+          tmem_st32(tS + 0, w);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(L::P_LO + x));
+        }
+        {
+          uint32_t w[32];
+          if (nvalid == kBN) exp_pack_half<true, 1>(s, m, sl2, acc, w);
+          else exp_pack_half<false, 1>(s, m, sl2, acc, w);
+          tmem_st32(tS + 32, w);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(L::P_HI + x));
         }
         l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-        tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&w[0]));
-        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&w[32]));
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(L::P_FULL + x));
         prev = p;
       }
     }
