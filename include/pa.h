@@ -153,6 +153,26 @@ typedef struct {
  * first need.  Errors: PA_EINVAL, PA_EALIGN, PA_EUNSUPPORTED, PA_ENOMEM, PA_ECUDA. */
 int pa_merge_states(pa_ctx* ctx, const pa_merge_desc* desc, void* stream);
 
+/* ---------------------------------------------------------------- merge without allocation */
+/* The same merge (and optional fused importance) as pa_merge_states, for callers that
+ * cannot allocate device memory: a process whose memory is owned by another allocator
+ * (a framework's caching pool holding the free HBM), or a latency-critical loop that must
+ * not stall, since cudaMalloc / cudaFree of a growing workspace synchronise the device.
+ * It takes no context (creating one allocates) and allocates nothing: its scratch is a
+ * fixed 4 MiB file-scope device array inside libpa, present on every GPU that loads the
+ * library until the process exits.  The pages describe no such variant; it has no
+ * counterpart there.
+ *
+ * Arguments, layouts and results are those of pa_merge_states.  The importance scratch
+ * needs P * B * H * sum over query groups of ceil(rows / 128) floats; larger requests
+ * return PA_EINVAL (use pa_merge_states).  The first call on a device looks up the
+ * scratch's device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture.  Every call shares the one scratch array, whose
+ * contents persist between calls (each call writes every scratch entry it reads, so none
+ * needs clearing): calls that overlap on the GPU -- on different streams, or from several
+ * threads -- race on it.  Errors go to pa_last_error(NULL). */
+int pa_merge_states_noalloc(const pa_merge_desc* desc, void* stream);
+
 /* ---------------------------------------------------------------- importance */
 /* w[qg][p] = mean over b, h and rows i of qg of exp(lse_part[p][b][h][i] - lse[b][h][i])
  * (0 where lse is -inf).  w is overwritten.  Same workspace rule as pa_merge_states.

@@ -8,6 +8,7 @@ names follow the C ABI in ``include/pa.h``:
 
     pa_init / Context            pa_partition_attn    pa_merge_states
     pa_importance                pa_relayout_seq2head pa_sync_status
+    pa_merge_states_noalloc
 
 There is no fallback: if ``libpa.so`` is missing or the device is not sm_100 the calls
 raise.
@@ -22,7 +23,7 @@ import numpy as np
 __all__ = [
     "PA_F32", "PA_BF16", "PAError", "Context", "lib", "lib_path",
     "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head",
-    "EXPORTED", "select_fresh",
+    "pa_merge_states_noalloc", "EXPORTED", "select_fresh",
 ]
 
 PA_F32, PA_BF16 = 0, 1
@@ -30,7 +31,8 @@ PA_MAX_P = 128
 _ERRORS = {-1: "PA_EINVAL", -2: "PA_EALIGN", -3: "PA_EUNSUPPORTED", -4: "PA_ENOMEM",
            -5: "PA_ECUDA", -6: "PA_ETIMEOUT"}
 EXPORTED = ("pa_init", "pa_destroy", "pa_last_error", "pa_sync_status", "pa_version",
-            "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head")
+            "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head",
+            "pa_merge_states_noalloc")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -86,9 +88,10 @@ def lib():
         L.pa_version.restype = ctypes.c_char_p
         L.pa_partition_attn.argtypes = [vp, ctypes.POINTER(_AttnDesc), vp]
         L.pa_merge_states.argtypes = [vp, ctypes.POINTER(_MergeDesc), vp]
+        L.pa_merge_states_noalloc.argtypes = [ctypes.POINTER(_MergeDesc), vp]
         L.pa_importance.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
         L.pa_relayout_seq2head.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, vp]
-        for f in ("pa_init", "pa_sync_status", "pa_partition_attn", "pa_merge_states",
+        for f in ("pa_init", "pa_sync_status", "pa_partition_attn", "pa_merge_states", "pa_merge_states_noalloc",
                   "pa_importance", "pa_relayout_seq2head"):
             getattr(L, f).restype = ci
         _LIB = L
@@ -189,6 +192,24 @@ def pa_merge_states(ctx: Context, part_off, G, fresh, o_fresh, lse_fresh, o_cach
                    None if fr is None else fr.ctypes.data, o.data_ptr(), lse.data_ptr(),
                    None if w is None else w.data_ptr())
     _check(ctx.ptr, lib().pa_merge_states(ctx.ptr, ctypes.byref(d), _stream(stream)))
+
+
+def pa_merge_states_noalloc(part_off, G, fresh, o_fresh, lse_fresh, o_cached, lse_cached, o, lse,
+                            w=None, stream=None):
+    """pa_merge_states without a context and without any device allocation: the fused
+    importance uses libpa's fixed 4 MiB scratch array (for callers that must not call
+    cudaMalloc).  Calls that overlap on the GPU share that scratch and must not be issued
+    concurrently."""
+    P, B, H, N, D = o_fresh.shape
+    off = _host_i32(part_off)
+    fr = _host_u8(fresh)
+    d = _MergeDesc(_dtype_code(o_fresh), B, H, N, D, P, int(G), off.ctypes.data,
+                   o_fresh.data_ptr(), lse_fresh.data_ptr(),
+                   None if o_cached is None else o_cached.data_ptr(),
+                   None if lse_cached is None else lse_cached.data_ptr(),
+                   None if fr is None else fr.ctypes.data, o.data_ptr(), lse.data_ptr(),
+                   None if w is None else w.data_ptr())
+    _check(None, lib().pa_merge_states_noalloc(ctypes.byref(d), _stream(stream)))
 
 
 def pa_importance(ctx: Context, part_off, G, lse_part, lse, w, stream=None):

@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "../../include/pa.h"
@@ -412,3 +413,113 @@ int pa_relayout_seq2head(pa_ctx* ctx, const void* src, void* dst, int N, int H, 
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ allocation-free merge
+// Scratch for pa_merge_states_noalloc: the per-block importance sums.  A file-scope device
+// array, so every GPU that loads this library holds it (4 MiB) until the process exits.
+// Host code must not use the symbol as a pointer: its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+namespace {
+
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;   // 4 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[128] = {};
+
+int noalloc_scratch(int device, float** out) {
+  if (device < 0 || device >= 128) return fail(nullptr, PA_EINVAL, "device %d outside [0, 128)", device);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[device]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return fail(nullptr, PA_ECUDA, "cudaGetSymbolAddress of the merge scratch failed on device %d: %s",
+                  device, cudaGetErrorString(e));
+    }
+    g_noalloc_ptr[device] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[device];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" int pa_merge_states_noalloc(const pa_merge_desc* d, void* stream) {
+  if (!d) return fail(nullptr, PA_EINVAL, "desc is NULL");
+  if (d->dtype != PA_BF16 && d->dtype != PA_F32) return fail(nullptr, PA_EUNSUPPORTED, "dtype %d", (int)d->dtype);
+  if (d->D != 64 && d->D != 128) return fail(nullptr, PA_EUNSUPPORTED, "D=%d (supported: 64, 128)", d->D);
+  if (d->B < 1 || d->H < 1 || d->N < 0) return fail(nullptr, PA_EINVAL, "B=%d H=%d N=%d", d->B, d->H, d->N);
+  const long long BH = static_cast<long long>(d->B) * d->H;
+  pa::AttnTables t;
+  int rc = build_tables(nullptr, d->N, d->P, d->G, d->part_off, d->fresh, t);
+  if (rc) return rc;
+  bool all_fresh = true;
+  for (int qg = 0; qg < t.QG; ++qg)
+    for (int p = 0; p < t.P; ++p) all_fresh &= pa::fresh_bit(t.fresh_bits, qg, p);
+  if (d->N == 0) return PA_OK;
+  if (!d->o_fresh || !d->lse_fresh || !d->o || !d->lse) return fail(nullptr, PA_EINVAL, "null tensor pointer");
+  if (!all_fresh && (!d->o_cached || !d->lse_cached))
+    return fail(nullptr, PA_EINVAL, "cached states are NULL but the mask reuses some pairs");
+  if (!aligned(d->o_fresh, 16) || !aligned(d->o, 16) || (d->o_cached && !aligned(d->o_cached, 16)))
+    return fail(nullptr, PA_EALIGN, "o_fresh, o_cached and o must be 16-byte aligned");
+  if (!aligned(d->lse_fresh, 4) || !aligned(d->lse, 4) || (d->lse_cached && !aligned(d->lse_cached, 4)) ||
+      (d->w && !aligned(d->w, 4)))
+    return fail(nullptr, PA_EALIGN, "lse arrays and w must be 4-byte aligned");
+  pa::MergeParams prm;
+  memset(&prm, 0, sizeof prm);
+  const int bpb = fill_blk_start(t, prm.blk_start);
+  const long long blocks = BH * bpb;
+  if (blocks > 0x7fffffffLL) return fail(nullptr, PA_EINVAL, "too many row blocks");
+  float* scratch = nullptr;
+  if (d->w) {
+    const unsigned long long need = static_cast<unsigned long long>(blocks) * t.P;
+    if (need > kNoAllocScratchFloats)
+      return fail(nullptr, PA_EINVAL,
+                  "importance scratch of %llu floats exceeds the fixed %zu (B*H*ceil(rows/128 per query "
+                  "group)*P); use pa_merge_states",
+                  need, kNoAllocScratchFloats);
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(nullptr, PA_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if ((rc = noalloc_scratch(dev, &scratch))) return rc;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  prm.o_fresh = d->o_fresh;
+  prm.lse_fresh = d->lse_fresh;
+  prm.o_cached = d->o_cached;
+  prm.lse_cached = d->lse_cached;
+  prm.o = d->o;
+  prm.lse = d->lse;
+  prm.w_partial = scratch;
+  prm.BH = (int)BH;
+  prm.N = d->N;
+  prm.D = d->D;
+  prm.P = t.P;
+  prm.G = t.G;
+  prm.QG = t.QG;
+  prm.blocks_per_bh = bpb;
+  memcpy(prm.part_off, t.part_off, sizeof prm.part_off);
+  memcpy(prm.qg_row0, t.qg_row0, sizeof prm.qg_row0);
+  memcpy(prm.fresh_bits, t.fresh_bits, sizeof prm.fresh_bits);
+  int e = pa::launch_merge(prm, d->dtype, st);
+  if (e) return fail(nullptr, PA_ECUDA, "merge launch: %s", cudaGetErrorString(static_cast<cudaError_t>(e)));
+  if (!d->w) return PA_OK;
+  pa::ReduceWParams r;
+  memset(&r, 0, sizeof r);
+  r.w_partial = scratch;
+  r.w = d->w;
+  r.BH = (int)BH;
+  r.P = t.P;
+  r.QG = t.QG;
+  r.blocks_per_bh = bpb;
+  for (int g = 0; g <= t.QG; ++g) r.blk_start[g] = prm.blk_start[g];
+  for (int g = 0; g < t.QG; ++g) {
+    const long long rows = t.qg_row0[g + 1] - t.qg_row0[g];
+    r.inv_count[g] = rows > 0 ? 1.0 / (static_cast<double>(rows) * BH) : 0.0;
+  }
+  e = pa::launch_reduce_w(r, st);
+  if (e) return fail(nullptr, PA_ECUDA, "reduce_w launch: %s", cudaGetErrorString(static_cast<cudaError_t>(e)));
+  return PA_OK;
+}
