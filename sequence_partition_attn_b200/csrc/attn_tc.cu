@@ -119,6 +119,16 @@ __device__ __forceinline__ float row_max128(const float (&s)[128]) {
   return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
 }
 
+// First key row of the 128-key box loaded for the tile that starts at `key` in partition
+// [k0, k1).  A partial last tile of a partition with at least 128 keys is loaded ending at
+// k1 (shifted back over keys already processed, which the softmax masks), so K and V rows
+// outside the partition are never read: masked keys get P = 0, and 0 * V is 0 only for
+// finite V -- rows of another partition may be non-finite or, in the chunked relayout
+// pipeline, still being written.  Partitions shorter than 128 keys load [k0, k0 + 128).
+__device__ __forceinline__ int tile_row0(int key, int k0, int k1) {
+  return (key + kBN > k1 && k1 - kBN >= k0) ? k1 - kBN : key;
+}
+
 // Next partition >= from that is fresh for query group qg and holds at least one key.
 __device__ __forceinline__ int next_part(const AttnTables& t, int qg, int from) {
   for (int p = from; p < t.P; ++p)
@@ -236,19 +246,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       bool ok = true;
       for (int p = next_part(t, qg, 0); ok && p < t.P; p = next_part(t, qg, p + 1)) {
         const int k1 = t.part_off[p + 1];
-        for (int key = t.part_off[p]; key < k1; key += kBN, ++j) {
+        const int k0 = t.part_off[p];
+        for (int key = k0; key < k1; key += kBN, ++j) {
           const int s = j % kStages;
           if (j >= kStages &&
               !mbar_wait(bar(L::KV_EMPTY + s), ((j / kStages) - 1) & 1, abort_flag, status)) {
             ok = false;
             break;
           }
+          const int ty = tile_row0(key, k0, k1);
           mbar_expect_tx(bar(L::K_FULL + s), L::kTileBytes);
           for (int a = 0; a < L::kAtoms; ++a)
-            tma_load_3d(sK(s) + a * kAtomBytes, &prm.tm_k, a * 64, key, bh, bar(L::K_FULL + s));
+            tma_load_3d(sK(s) + a * kAtomBytes, &prm.tm_k, a * 64, ty, bh, bar(L::K_FULL + s));
           mbar_expect_tx(bar(L::V_FULL + s), L::kTileBytes);
           for (int a = 0; a < L::kAtoms; ++a)
-            tma_load_3d(sV(s) + a * kAtomBytes, &prm.tm_v, a * 64, key, bh, bar(L::V_FULL + s));
+            tma_load_3d(sV(s) + a * kAtomBytes, &prm.tm_v, a * 64, ty, bh, bar(L::V_FULL + s));
         }
       }
       // Every load issued must have landed before the CTA may exit.
@@ -411,8 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         const int nvalid = min(kBN, k1 - key);
         if (nvalid < kBN) {
+          // Keys outside [key, k1) of the loaded box: the leading ones of a shifted last
+          // tile (already processed), or the trailing ones of a partition shorter than a tile.
+          const int lo = tile_row0(key, k0, k1) < key ? kBN - nvalid : 0;
 #pragma unroll
-          for (int c = 0; c < kBN; ++c) s[c] = c < nvalid ? s[c] : -INFINITY;
+          for (int c = 0; c < kBN; ++c) s[c] = (c >= lo && c < lo + nvalid) ? s[c] : -INFINITY;
         }
         const float mt = row_max128(s) * sl2;
         if (key == k0) {

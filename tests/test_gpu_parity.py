@@ -227,3 +227,27 @@ def test_empty_sequence_is_a_no_op(pa, ctx):
     l = torch.zeros(1, 1, 1, 0, device=DEV)
     pa.pa_partition_attn(ctx, q, q, q, [0, 0], 1, None, o, l)
     ctx.sync_status()
+
+
+def test_partition_state_reads_no_other_partition(pa, ctx):
+    # A partition of >= 128 keys must not depend on K/V rows of any other partition, even
+    # non-finite ones (its last partial tile is loaded ending at the partition end).
+    wl = W.small_variant(W.workload(1), grid=(1, 25, 40), H=2, P=4, G=1, mask="all")   # 250 keys each
+    t = W.make_qkv(wl)
+    off = W.part_offsets(wl.N, wl.P)
+    q, k, v = (t[n].to(DEV) for n in ("q", "k", "v"))
+    fresh = np.zeros((4, 4), dtype=np.uint8)
+    fresh[:, 1] = 1                                              # every query group x partition 1
+    o1 = torch.zeros(4, 1, 2, wl.N, 128, dtype=torch.bfloat16, device=DEV)
+    l1 = torch.zeros(4, 1, 2, wl.N, device=DEV)
+    pa.pa_partition_attn(ctx, q, k, v, off, 1, fresh, o1, l1)
+    k2, v2 = k.clone(), v.clone()
+    for p in (0, 2, 3):
+        k2[:, :, off[p]:off[p + 1]] = float("nan")
+        v2[:, :, off[p]:off[p + 1]] = float("inf")
+    o2 = torch.zeros_like(o1)
+    l2 = torch.zeros_like(l1)
+    pa.pa_partition_attn(ctx, q, k2, v2, off, 1, fresh, o2, l2)
+    ctx.sync_status()
+    assert torch.isfinite(o2[1].float()).all() and torch.isfinite(l2[1]).all()
+    assert torch.equal(o1[1].view(torch.int16), o2[1].view(torch.int16)) and torch.equal(l1[1], l2[1])
