@@ -340,6 +340,8 @@ def run_ours(args, ws, rank, local):
     extras = {}
     if not args.no_extras:
         wl4 = W.workload(4)
+        if args.workload == "720p-small":          # 2 of 16 chunks' worth: 4 chunks, 16 partitions
+            wl4 = W.small_variant(wl4, grid=(2, 90, 160), H=wl4.H, P=16, chunks=4)
         N4, H4, D4 = wl4.N, wl4.H, wl4.D
         srcs = [torch.empty(N4, H4, D4, dtype=torch.bfloat16, device=dev).normal_() for _ in range(3)]
         dsts = [torch.empty(1, H4, N4, D4, dtype=torch.bfloat16, device=dev) for _ in range(3)]

@@ -34,7 +34,7 @@
 // touch O_x after waiting only for S_x(j+1).
 //
 // Exponentials: 2^t on full tiles can be split between the MUFU unit and a degree-3
-// polynomial on the FMA pipe (kPolyCols of every 8 columns): Cody-Waite split t = n + f,
+// polynomial on the FMA pipe (kPolyPairs of every 8 column pairs): Cody-Waite split t = n + f,
 // |f| <= 1/2, 2^f by a minimax polynomial fitted for this kernel (fit_exp2_poly.py, max
 // relative error 7.5e-5), 2^n added to the exponent field.
 #include "pa_device.cuh"
@@ -60,9 +60,9 @@ struct Layout {
   static constexpr int kK = kQ + 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
   static constexpr int kBar = kV + kStages * kTileBytes;
-  enum { Q_FULL = 0, K_FULL = 1, V_FULL = K_FULL + kStages, KV_EMPTY = V_FULL + kStages,
-         S_FULL = KV_EMPTY + kStages, P_LO = S_FULL + 2, P_HI = P_LO + 2, O_DONE = P_HI + 2,
-         NBAR = O_DONE + 2 };
+  enum { Q_FULL = 0, K_FULL = 1, V_FULL = K_FULL + kStages, K_EMPTY = V_FULL + kStages,
+         V_EMPTY = K_EMPTY + kStages, S_FULL = V_EMPTY + kStages, P_LO = S_FULL + 2, P_HI = P_LO + 2,
+         O_DONE = P_HI + 2, NBAR = O_DONE + 2 };
   static constexpr int kTmemSlot = kBar + NBAR * 8;
   static constexpr int kAbort = kTmemSlot + 8;
   static constexpr int kUsed = kAbort + 8;
@@ -73,14 +73,11 @@ struct Layout {
 
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;    // move the running max only when it grows by > 8
-// Columns out of every 8 whose exponential runs on the FMA pipe (polynomial) instead of
-// MUFU.  Measured on B200 at the 720p shape: 0 -> 893, 1 -> 891, 2 -> 859, 3 -> 817,
-// 4 -> 779 TFLOP/s, so the MUFU unit is not the limiter of this kernel and all
-// exponentials go to it.
-constexpr int kPolyCols = 0;
-// true: the MMA issuer polls the softmax hand-off barriers (test_wait) instead of sleeping
-// on them (try_wait).  Measured at the 720p shape: no difference beyond run-to-run noise.
-constexpr bool kPollHandoff = false;
+// Column pairs out of every 8 whose exponentials run on the FMA pipe (packed polynomial)
+// instead of MUFU, on tiles with every key valid.  Measured at the 720p shape (packed
+// scale/sum in place): 0 -> 1010, 1 -> 998, 2 -> 962, 3 -> 955, 4 -> 921 TFLOP/s, so all
+// exponentials go to MUFU.
+constexpr int kPolyPairs = 0;
 
 // Minimax coefficients of 2^f on [-1/2, 1/2] (relative error), from fit_exp2_poly.py.
 constexpr float kC0 = 0.9999280571937561f;
@@ -129,6 +126,21 @@ __device__ __forceinline__ int tile_row0(int key, int k0, int k1) {
   return (key + kBN > k1 && k1 - kBN >= k0) ? k1 - kBN : key;
 }
 
+// The same on a pair of values with packed fp32x2 arithmetic (one instruction per pair
+// for the rounding, the reduction and the polynomial).
+__device__ __forceinline__ float2 poly_exp2x2(float2 t) {
+  t.x = fmaxf(t.x, -126.0f);
+  t.y = fmaxf(t.y, -126.0f);
+  const float2 rnd = __fadd2_rn(t, make_float2(12582912.0f, 12582912.0f));
+  const float2 n = __fadd2_rn(rnd, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __fadd2_rn(t, make_float2(-n.x, -n.y));
+  float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+  p = __ffma2_rn(p, f, make_float2(kC0, kC0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(rnd.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(rnd.y) << 23)));
+}
+
 // Next partition >= from that is fresh for query group qg and holds at least one key.
 __device__ __forceinline__ int next_part(const AttnTables& t, int qg, int from) {
   for (int p = from; p < t.P; ++p)
@@ -148,13 +160,16 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 }
 
 // S_x = Q_x K^T: D/16 MMAs of 128 x 128 x 16 (K-major operands, 128-byte swizzle; the
-// k-step moves 32 bytes inside a 64-element swizzle atom, then to the next atom).
+// k-step moves 32 bytes inside a 64-element swizzle atom, then to the next atom).  Called
+// by a whole warp: operands stay warp-uniform and one elected lane issues each MMA (an
+// issue path divergent on one lane costs ~50 cycles per MMA, a uniform one ~17-21).
 template <int D>
 __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t dq, uint64_t dk, uint32_t idesc) {
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = static_cast<uint32_t>(((kk >> 2) * kAtomBytes + (kk & 3) * 32) >> 4);
-    mma_bf16_ss(d_tmem, dq + off, dk + off, idesc, kk > 0);
+    if (elect_one()) mma_bf16_ss(d_tmem, dq + off, dk + off, idesc, kk > 0);
+    __syncwarp();
   }
 }
 
@@ -165,25 +180,36 @@ template <int D, int H>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t dv, uint32_t idesc,
                                          bool first) {
 #pragma unroll
-  for (int kk = H * 4; kk < H * 4 + 4; ++kk)
-    mma_bf16_ts(d_tmem, p_tmem + kk * 8, dv + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc,
-                (first && kk == 0) ? 0u : 1u);
+  for (int kk = H * 4; kk < H * 4 + 4; ++kk) {
+    if (elect_one())
+      mma_bf16_ts(d_tmem, p_tmem + kk * 8, dv + static_cast<uint32_t>((kk * 16 * 128) >> 4), idesc,
+                  (first && kk == 0) ? 0u : 1u);
+    __syncwarp();
+  }
 }
 
-// Exponentials of half H of a row (columns 64H .. 64H+63), added to the 8 row-sum chains
-// and packed to bf16 pairs (32 TMEM columns).  kFull: every key valid (masked keys hold
-// -inf otherwise, and MUFU's exp2(-inf) = 0 handles them).
+// Exponentials of half H of a row (columns 64H .. 64H+63), added to the row-sum chains
+// and packed to bf16 pairs (32 TMEM columns).  Scale-and-shift and the sums use Blackwell's
+// packed fp32x2 FMA / ADD (one instruction per pair).  kFull: every key valid (masked keys
+// hold -inf otherwise, and MUFU's exp2(-inf) = 0 handles them).
 template <bool kFull, int H>
-__device__ __forceinline__ void exp_pack_half(const float (&s)[128], float m, float sl2, float (&acc)[8],
+__device__ __forceinline__ void exp_pack_half(const float (&s)[128], float m, float sl2, float2 (&acc)[4],
                                               uint32_t (&w)[32]) {
+  const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-m, -m);
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const int c = H * 64 + 2 * i;
-    const float a0 = fmaf(s[c], sl2, -m), a1 = fmaf(s[c + 1], sl2, -m);
-    const float e0 = (kFull && (c & 7) >= 8 - kPolyCols) ? poly_exp2(a0) : fast_exp2(a0);
-    const float e1 = (kFull && ((c + 1) & 7) >= 8 - kPolyCols) ? poly_exp2(a1) : fast_exp2(a1);
-    acc[c & 7] += e0;
-    acc[(c + 1) & 7] += e1;
+    const float2 a = __ffma2_rn(make_float2(s[c], s[c + 1]), scale2, neg_m2);
+    float e0, e1;
+    if (kFull && (i & 7) < kPolyPairs) {
+      const float2 e = poly_exp2x2(a);
+      e0 = e.x;
+      e1 = e.y;
+    } else {
+      e0 = fast_exp2(a.x);
+      e1 = fast_exp2(a.y);
+    }
+    acc[i & 3] = __fadd2_rn(acc[i & 3], make_float2(e0, e1));
     w[i] = pack_bf16x2(e0, e1);
   }
 }
@@ -249,15 +275,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const int k0 = t.part_off[p];
         for (int key = k0; key < k1; key += kBN, ++j) {
           const int s = j % kStages;
-          if (j >= kStages &&
-              !mbar_wait(bar(L::KV_EMPTY + s), ((j / kStages) - 1) & 1, abort_flag, status)) {
+          const uint32_t ph = ((j / kStages) - 1) & 1;
+          const int ty = tile_row0(key, k0, k1);
+          // K's slot frees when both S products that read it complete, V's when both PV
+          // products do: K runs a tile ahead of V.
+          if (j >= kStages && !mbar_wait(bar(L::K_EMPTY + s), ph, abort_flag, status)) {
             ok = false;
             break;
           }
-          const int ty = tile_row0(key, k0, k1);
           mbar_expect_tx(bar(L::K_FULL + s), L::kTileBytes);
           for (int a = 0; a < L::kAtoms; ++a)
             tma_load_3d(sK(s) + a * kAtomBytes, &prm.tm_k, a * 64, ty, bh, bar(L::K_FULL + s));
+          if (j >= kStages && !mbar_wait(bar(L::V_EMPTY + s), ph, abort_flag, status)) {
+            ok = false;
+            break;
+          }
           mbar_expect_tx(bar(L::V_FULL + s), L::kTileBytes);
           for (int a = 0; a < L::kAtoms; ++a)
             tma_load_3d(sV(s) + a * kAtomBytes, &prm.tm_v, a * 64, ty, bh, bar(L::V_FULL + s));
@@ -272,7 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // Whole warp, warp-uniform control flow; one elected lane issues each MMA and commit.
+    {
       constexpr uint32_t kIdS = idesc_bf16(kBM, kBN, false, false);   // Q K-major, K K-major
       constexpr uint32_t kIdPV = idesc_bf16(kBM, D, false, true);     // P (TMEM), V MN-major
       int T = 0;
@@ -286,20 +319,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint64_t dk1 = smem_desc_sw128(sK(1), 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(sV(0), kAtomBytes, 1024);
       const uint64_t dv1 = smem_desc_sw128(sV(1), kAtomBytes, 1024);
-      auto wait_p = [&](uint32_t b, uint32_t parity) {
-        return kPollHandoff ? mbar_wait_poll(b, parity, abort_flag, status)
-                            : mbar_wait(b, parity, abort_flag, status);
+      auto commit = [&](int b) {
+        if (elect_one()) mma_commit(bar(b));
+        __syncwarp();
       };
-      bool ok = mbar_wait(bar(L::Q_FULL), 0, abort_flag, status);
+      auto wait_p = [&](uint32_t b, uint32_t parity) { return mbar_wait_warp(b, parity, abort_flag, status); };
+      bool ok = mbar_wait_warp(bar(L::Q_FULL), 0, abort_flag, status);
       int j = 0;
       if (ok && T > 0) {
-        ok = mbar_wait(bar(L::K_FULL + 0), 0, abort_flag, status);
+        ok = mbar_wait_warp(bar(L::K_FULL + 0), 0, abort_flag, status) &&
+             mbar_wait_warp(bar(L::V_FULL + 0), 0, abort_flag, status);
         if (ok) {
           tc_fence_after();
           issue_s<D>(tmem, dq0, dk0, kIdS);
-          mma_commit(bar(L::S_FULL + 0));
+          commit(L::S_FULL + 0);
           issue_s<D>(tmem + 128, dq1, dk0, kIdS);
-          mma_commit(bar(L::S_FULL + 1));
+          commit(L::S_FULL + 1);
+          commit(L::K_EMPTY + 0);
         }
         int p = next_part(t, qg, 0);
         int key = t.part_off[p];
@@ -309,34 +345,40 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const bool more = j + 1 < T;
           const uint64_t dv = s ? dv1 : dv0;
           const uint64_t dk = s1 ? dk1 : dk0;
-          // Operand waits first (normally already complete), then the softmax hand-offs.
-          if (!mbar_wait(bar(L::V_FULL + s), (j / kStages) & 1, abort_flag, status)) { ok = false; break; }
-          if (more && !mbar_wait(bar(L::K_FULL + s1), ((j + 1) / kStages) & 1, abort_flag, status)) {
-            ok = false;
-            break;
-          }
+          // V(j) was waited for during the previous tile (or before the loop); operand
+          // waits sit where products are already queued, off the hand-off path.
           if (!wait_p(bar(L::P_LO + 0), j & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv<D, 0>(tmem + 256, tmem, dv, kIdPV, first);
           if (!wait_p(bar(L::P_HI + 0), j & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv<D, 1>(tmem + 256, tmem, dv, kIdPV, first);
-          mma_commit(bar(L::O_DONE + 0));
+          commit(L::O_DONE + 0);
           if (more) {
+            if (!mbar_wait_warp(bar(L::K_FULL + s1), ((j + 1) / kStages) & 1, abort_flag, status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
             issue_s<D>(tmem, dq0, dk, kIdS);
-            mma_commit(bar(L::S_FULL + 0));
+            commit(L::S_FULL + 0);
           }
           if (!wait_p(bar(L::P_LO + 1), j & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv<D, 0>(tmem + 384, tmem + 128, dv, kIdPV, first);
+          if (more && !mbar_wait_warp(bar(L::V_FULL + s1), ((j + 1) / kStages) & 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
           if (!wait_p(bar(L::P_HI + 1), j & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv<D, 1>(tmem + 384, tmem + 128, dv, kIdPV, first);
-          mma_commit(bar(L::O_DONE + 1));
-          mma_commit(bar(L::KV_EMPTY + s));
+          commit(L::O_DONE + 1);
+          commit(L::V_EMPTY + s);
           if (more) {
             issue_s<D>(tmem + 128, dq1, dk, kIdS);
-            mma_commit(bar(L::S_FULL + 1));
+            commit(L::S_FULL + 1);
+            commit(L::K_EMPTY + s1);
           }
           key += kBN;
           if (key >= t.part_off[p + 1]) {
@@ -346,8 +388,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
       }
       // The last commits must have arrived before the CTA may exit.
-      for (int jj = (j > kStages ? j - kStages : 0); jj < j; ++jj)
-        mbar_drain(bar(L::KV_EMPTY + jj % kStages), (jj / kStages) & 1);
+      if (lane == 0) {
+        for (int jj = (j > kStages ? j - kStages : 0); jj < j; ++jj) {
+          mbar_drain(bar(L::K_EMPTY + jj % kStages), (jj / kStages) & 1);
+          mbar_drain(bar(L::V_EMPTY + jj % kStages), (jj / kStages) & 1);
+        }
+      }
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- softmax warpgroups
@@ -453,7 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // Exponentials, row sum (8 independent chains) and P packed to bf16 pairs, half a
         // row at a time; each half of P goes over S_x's first 64 columns and is handed to
         // the MMA issuer at once, so PV on keys 0-63 overlaps the exponentials of 64-127.
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
         {
           uint32_t w[32];
           if (nvalid == kBN) exp_pack_half<true, 0>(s, m, sl2, acc, w);
@@ -472,7 +519,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           tc_fence_before();
           mbar_arrive(bar(L::P_HI + x));
         }
-        l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        {
+          const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+          const float2 a = __fadd2_rn(a01, a23);
+          l += a.x + a.y;
+        }
         prev = p;
       }
     }
