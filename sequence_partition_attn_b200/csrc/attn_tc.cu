@@ -482,7 +482,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           m = mt;
           l = 0.0f;
         } else if (__any_sync(0xffffffffu, mt - m > kRescaleLog2)) {
-          const float m_new = fmaxf(m, mt);
+          // Only rows whose own max grew past the bound move it (alpha = 1 elsewhere), so
+          // a row's result never depends on which rows share its warp.
+          const float m_new = mt - m > kRescaleLog2 ? mt : m;
           const float alpha = fast_exp2(m - m_new);
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {

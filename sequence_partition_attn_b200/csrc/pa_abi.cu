@@ -86,6 +86,23 @@ int build_tables(pa_ctx* ctx, int N, int P, int G, const int32_t* part_off, cons
   return PA_OK;
 }
 
+// Attention tiling: consecutive query groups that select the same fresh partitions form
+// one segment, tiled as a unit (a row's states depend only on its own query and the
+// partitions computed for it, so tiles may straddle such groups).  Replaces the group
+// bounds and masks of `t` by the segments'.
+void merge_equal_groups(pa::AttnTables& t) {
+  int n = 0;
+  for (int g = 0; g < t.QG; ++g) {
+    if (n > 0 && memcmp(t.fresh_bits[n - 1], t.fresh_bits[g], sizeof t.fresh_bits[0]) == 0) continue;
+    if (n != g) memcpy(t.fresh_bits[n], t.fresh_bits[g], sizeof t.fresh_bits[0]);
+    t.qg_row0[n] = t.qg_row0[g];
+    ++n;
+  }
+  t.qg_row0[n] = t.qg_row0[t.QG];
+  for (int g = n; g < t.QG; ++g) memset(t.fresh_bits[g], 0, sizeof t.fresh_bits[0]);
+  t.QG = n;
+}
+
 // Prefix of row tiles over the query groups that have at least one fresh pair.
 int fill_tile_start(pa::AttnTables& t, int tile_rows) {
   int acc = 0;
@@ -255,6 +272,7 @@ int pa_partition_attn(pa_ctx* ctx, const pa_attn_desc* d, void* stream) {
     pa::TcParams prm;
     memset(&prm, 0, sizeof prm);
     prm.t = t;
+    merge_equal_groups(prm.t);
     const int tiles = fill_tile_start(prm.t, pa::attn_tc_tile_rows());
     if (tiles == 0) return PA_OK;
     if ((rc = encode_qkv_map(ctx, &prm.tm_q, d->q, (int)BH, d->N, d->D))) return rc;
@@ -276,6 +294,7 @@ int pa_partition_attn(pa_ctx* ctx, const pa_attn_desc* d, void* stream) {
   pa::F32AttnParams prm;
   memset(&prm, 0, sizeof prm);
   prm.t = t;
+  merge_equal_groups(prm.t);
   const int tiles = fill_tile_start(prm.t, pa::attn_f32_tile_rows());
   if (tiles == 0) return PA_OK;
   prm.q = static_cast<const float*>(d->q);

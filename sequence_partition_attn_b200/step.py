@@ -132,14 +132,17 @@ class Trajectory:
 
 
 def relayout_overlapped(ctx, src_qkv, dst_qkv, n_chunks, part_off, G, o_part, lse_part,
-                        s_copy, s_attn):
+                        s_copy, s_attn, milestones=None):
     """Chunked seq-major -> head-major relayout of Q, K, V on one stream, overlapped with
     partition attention over the chunks already moved on another (SwiftFusion web summary,
     Methodology 2, Torus Attention).  All pairs fresh.
 
-    Chunk c is relayed out (3 launches) and recorded; the attention stream waits for it and
-    computes the new pairs: query chunk c against KV chunks <= c, and query chunks < c
-    against KV chunk c.  Chunk boundaries must be partition boundaries.
+    Every chunk is relayed out on ``s_copy`` (3 launches) and recorded.  Attention runs in
+    a few launches at the chunk counts in ``milestones`` (default 1, 2, 4, ... n_chunks):
+    after chunks [0, m) have moved, it computes every (query chunk, KV chunk) pair whose
+    later chunk lies in [previous milestone, m).  Geometric milestones keep the first
+    attention launch early and the number of partially filled launches small.  Chunk
+    boundaries must be group boundaries.  Returns the relayout events.
     """
     src_q, src_k, src_v = src_qkv
     q, k, v = dst_qkv
@@ -148,6 +151,12 @@ def relayout_overlapped(ctx, src_qkv, dst_qkv, n_chunks, part_off, G, o_part, ls
     assert per * n_chunks == P and per % G == 0
     QG = -(-P // G)
     gpc = per // G                          # groups per chunk
+    if milestones is None:
+        milestones, m = [], 1
+        while m < n_chunks:
+            milestones.append(m)
+            m *= 2
+        milestones.append(n_chunks)
     events = []
     for c in range(n_chunks):
         with torch.cuda.stream(s_copy):
@@ -157,10 +166,13 @@ def relayout_overlapped(ctx, src_qkv, dst_qkv, n_chunks, part_off, G, o_part, ls
             ev = torch.cuda.Event()
             ev.record(s_copy)
             events.append(ev)
-        s_attn.wait_event(ev)
+    prev = 0
+    for m in milestones:
+        s_attn.wait_event(events[m - 1])
         mask = np.zeros((QG, QG), dtype=np.uint8)
-        lo, hi = c * gpc, (c + 1) * gpc
-        mask[lo:hi, :hi] = 1                # query chunk c x KV chunks <= c
-        mask[:lo, lo:hi] = 1                # query chunks < c x KV chunk c
+        lo, hi = prev * gpc, m * gpc
+        mask[lo:hi, :hi] = 1                # new query chunks x every moved KV chunk
+        mask[:lo, lo:hi] = 1                # earlier query chunks x new KV chunks
         pa_partition_attn(ctx, q, k, v, part_off, G, mask, o_part, lse_part, stream=s_attn)
+        prev = m
     return events
