@@ -25,6 +25,10 @@ What is computed, and where the pages state it (DiTango web summary, Methodology
   anchor steps: importance is refreshed at anchors).
 * select_fresh -- the reuse decision from stored importance: a KV group is recomputed when
   any of its partitions has stored importance >= threshold.
+* compose_states / merge_with_composed_cache -- dynamic group compose (DiTango web summary,
+  Methodology 2 "Dynamic Group Compose"): cached states of consecutive partitions merge
+  into one coarser state with no recomputation, and a reused KV group then contributes
+  its single composed state to the merge.
 * relayout_seq2head -- the sequence-major -> head-major permutation that the Ulysses
   all-to-all performs, here on one device (SwiftFusion, Methodology 2).
 
@@ -41,7 +45,8 @@ import numpy as np
 
 __all__ = [
     "partition_states", "merge_states", "merge_with_reuse", "importance",
-    "select_fresh", "relayout_seq2head", "group_bounds",
+    "select_fresh", "relayout_seq2head", "group_bounds", "compose_states",
+    "merge_with_composed_cache",
 ]
 
 
@@ -134,6 +139,45 @@ def merge_with_reuse(o_fresh, lse_fresh, o_cached, lse_cached, part_off, G, fres
         o_sel.append(np.where(use_fresh[None, None, :, None], o_fresh[p], o_cached[p]))
     O, L = merge_states(o_sel, l_sel)
     return O, L, np.stack(l_sel, axis=0)
+
+
+def compose_states(o_part, lse_part, factor):
+    """Merge the states of every `factor` consecutive partitions into one.
+
+    o_part [P, ...rows, D], lse_part [P, ...rows] -> ([ceil(P/factor), ...], [...]); group c
+    is the composition of partitions c*factor .. min((c+1)*factor, P) - 1.
+    """
+    P = lse_part.shape[0]
+    C = -(-P // factor)
+    outs = [merge_states(list(o_part[c * factor:(c + 1) * factor]),
+                         list(lse_part[c * factor:(c + 1) * factor])) for c in range(C)]
+    return np.stack([o for o, _ in outs]), np.stack([l for _, l in outs])
+
+
+def merge_with_composed_cache(o_fresh, lse_fresh, o_comp, lse_comp, part_off, G, fresh, rows=None):
+    """Merge per row: for KV group kg, the fresh per-partition states of its partitions when
+    fresh[qg, kg], else its one composed cached state o_comp[kg], lse_comp[kg].
+
+    o_fresh [P, B, H, R, D]; o_comp [KG, B, H, R, D].  Returns (O, LSE).
+    """
+    P = len(part_off) - 1
+    KG = -(-P // G)
+    R = lse_fresh.shape[-1]
+    rows = np.arange(R) if rows is None else np.asarray(rows)
+    qg_of_row = _row_groups(rows, part_off, G)
+    o_sel, l_sel = [], []
+    for kg in range(KG):
+        use_fresh = (fresh[qg_of_row, kg] != 0)                       # [R]
+        for p in range(kg * G, min((kg + 1) * G, P)):
+            if p == kg * G:
+                # the group's first slot carries the cached state where reused
+                l_sel.append(np.where(use_fresh[None, None, :], lse_fresh[p], lse_comp[kg]))
+                o_sel.append(np.where(use_fresh[None, None, :, None], o_fresh[p], o_comp[kg]))
+            else:
+                # further partitions only where fresh; reused rows take nothing (-inf)
+                l_sel.append(np.where(use_fresh[None, None, :], lse_fresh[p], -np.inf))
+                o_sel.append(np.where(use_fresh[None, None, :, None], o_fresh[p], 0.0))
+    return merge_states(o_sel, l_sel)
 
 
 def importance(lse_part, lse, part_off, G, rows=None):

@@ -430,3 +430,36 @@ def test_spatial_locality_of_the_generated_inputs():
     for g in range(wl.P):
         far = 0 if g >= wl.P // 2 else wl.P - 1
         assert w[g, g] > w[g, far]
+
+
+# --------------------------------------------------------------------------- group compose
+def test_composed_cache_equals_per_partition_cache():
+    # Dynamic group compose (DiTango, Methodology 2): composing cached states per group and
+    # merging the composed ones gives the same result as merging the per-partition cache.
+    q, k, v = rand_qkv(21, 1, 2, 70, 8)
+    P, G = 6, 3
+    off = W.part_offsets(70, P)
+    ones = all_fresh(P, G)
+    of, lf, _ = O.partition_states(q, k, v, off, G, ones, 0.35)
+    rng = np.random.default_rng(22)
+    kc, vc = k + 0.2 * rng.standard_normal(k.shape), v + 0.2 * rng.standard_normal(v.shape)
+    oc, lc, _ = O.partition_states(q, kc, vc, off, G, ones, 0.35)
+    fresh = np.array([[1, 0], [0, 1]], dtype=np.uint8)
+    ref_o, ref_l, _ = O.merge_with_reuse(of, lf, oc, lc, off, G, fresh)
+    co, cl = O.compose_states(oc, lc, G)
+    assert co.shape[0] == 2
+    o, l = O.merge_with_composed_cache(of, lf, co, cl, off, G, fresh)
+    np.testing.assert_allclose(o, ref_o, atol=1e-12)
+    np.testing.assert_allclose(l, ref_l, atol=1e-12)
+
+
+def test_composed_state_is_attention_over_the_group():
+    # a composed group state equals the state of one partition spanning the whole group
+    q, k, v = rand_qkv(23, 1, 1, 40, 4)
+    off = W.part_offsets(40, 4)                  # 10 keys each
+    ones = all_fresh(4)
+    op, lp, _ = O.partition_states(q, k, v, off, 1, ones, 0.5)
+    co, cl = O.compose_states(op, lp, 2)
+    wide, wl, _ = O.partition_states(q, k, v, np.array([0, 20, 40]), 1, all_fresh(2), 0.5)
+    np.testing.assert_allclose(co, wide, atol=1e-12)
+    np.testing.assert_allclose(cl, wl, atol=1e-12)
