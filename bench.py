@@ -333,6 +333,44 @@ def run_ours(args, ws, rank, local):
         e2e = {"value": ws * step.flops * K / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K}
         del hq, hk, hv, ho, hl, hw
+    # ---- dynamic group compose: the cache composed per KV group, merged without importance
+    if not args.no_extras and step.o_cached is not None:
+        B, H, N, D, G, KG = wl.B, wl.H, wl.N, wl.D, wl.G, wl.KG
+        ocg = torch.empty(KG, B, H, N, D, dtype=torch.bfloat16, device=dev)
+        lcg = torch.empty(KG, B, H, N, dtype=torch.float32, device=dev)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pa.pa_compose_states(ctx, step.o_cached, step.lse_cached, G, ocg, lcg)
+        c0.record(stream)
+        pa.pa_compose_states(ctx, step.o_cached, step.lse_cached, G, ocg, lcg)
+        c1.record(stream)
+        for _ in range(3):
+            pa.pa_merge_states(ctx, off, G, fresh, step.o_fresh, step.lse_fresh, ocg, lcg, step.o,
+                               step.lse, cached_per_group=True)
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        m0.record(stream)
+        for _ in range(reps):
+            pa.pa_merge_states(ctx, off, G, fresh, step.o_fresh, step.lse_fresh, ocg, lcg, step.o,
+                               step.lse, cached_per_group=True)
+        m1.record(stream)
+        torch.cuda.synchronize()
+        ctx.sync_status()
+        gb = W.group_row_bounds(off, G)
+        row_b = D * 2 + 4
+        states = sum(int(gb[qg + 1] - gb[qg]) * sum(G if fresh[qg, kg] else 1 for kg in range(KG))
+                     for qg in range(wl.QG))
+        cm_bytes = float(B * H) * (states * row_b + N * row_b)
+        cm_ms = m0.elapsed_time(m1) / reps
+        cp_ms = c0.elapsed_time(c1)
+        compose_bytes = float(B * H * N) * row_b * (wl.P + KG)
+        composed_extra = {"merge_composed_cache": {"ms": cm_ms, "gbs": cm_bytes / (cm_ms / 1e3) / 1e9,
+                                                   "bytes": cm_bytes},
+                          "compose_cache": {"ms": cp_ms, "gbs": compose_bytes / (cp_ms / 1e3) / 1e9,
+                                            "cache_bytes_before": float(B * H * N) * row_b * wl.P,
+                                            "cache_bytes_after": float(B * H * N) * row_b * KG}}
+        del ocg, lcg
+    else:
+        composed_extra = {}
     del step
     torch.cuda.empty_cache()
 
@@ -403,7 +441,7 @@ def run_ours(args, ws, rank, local):
         "kernels": {"partition_attn": {"ms": attn_ms, "tflops": attn_tflops, "flops": step_flops},
                     "merge_importance": {"ms": merge_ms, "gbs": merge_gbs,
                                          "frac_of_hbm": merge_gbs / pk["hbm_gbs"]},
-                    **extras},
+                    **composed_extra, **extras},
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": attn_tflops / pk["bf16_tflops"],
                      "traffic": traffic, "peak_kind": f"{pk_kind} burst bf16",

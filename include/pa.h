@@ -144,14 +144,33 @@ typedef struct {
   void* o;                   /* [B][H][N][D] out */
   float* lse;                /* [B][H][N]    out */
   float* w;                  /* [QG][P] out (fused importance of the merged states), or NULL */
+  int cached_per_group;      /* 0: o_cached / lse_cached hold per-partition states [P][..];
+                                1: they hold one composed state per KV group [KG][B][H][N](D)
+                                (see pa_compose_states); w must then be NULL */
 } pa_merge_desc;
 
 /* Per row i of query group qg: take the state of partition p from the fresh arrays when
  * fresh[qg][p/G] != 0, else from the cached arrays; write LSE(i), O(i) (fp32 math, O
  * rounded to dtype) and, if w != NULL, overwrite w with the importance of the merged
- * states.  Uses a context workspace of about 4*P*ceil(B*H*N/256) bytes, allocated on
+ * states.  With cached_per_group, a reused KV group contributes its one composed cached
+ * state instead of G per-partition states (fewer bytes read per row).  Uses a context workspace of about 4*P*ceil(B*H*N/256) bytes, allocated on
  * first need.  Errors: PA_EINVAL, PA_EALIGN, PA_EUNSUPPORTED, PA_ENOMEM, PA_ECUDA. */
 int pa_merge_states(pa_ctx* ctx, const pa_merge_desc* desc, void* stream);
+
+/* ---------------------------------------------------------------- group compose */
+/* Dynamic group compose of cached states (DiTango web summary, Methodology 2, "Dynamic
+ * Group Compose": cached states merge recursively into coarser groups with no
+ * recomputation).  For every row and every group c of `factor` consecutive partitions,
+ * writes the composition of their states: lse_group[c] = ln sum_p exp(lse_part[p]),
+ * o_group[c] = sum_p exp(lse_part[p] - lse_group[c]) o_part[p].
+ *   o_part [P][B][H][N][D], lse_part [P][B][H][N] in; o_group [C][B][H][N][D],
+ *   lse_group [C][B][H][N] out, C = ceil(P / factor).  Partitions of empty state
+ *   (-inf) contribute nothing.  Composing G partitions per group gives the cache that
+ *   pa_merge_states reads with cached_per_group = 1.
+ * Errors: PA_EINVAL, PA_EALIGN, PA_EUNSUPPORTED, PA_ECUDA. */
+int pa_compose_states(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int P, int factor,
+                      const void* o_part, const float* lse_part, void* o_group, float* lse_group,
+                      void* stream);
 
 /* ---------------------------------------------------------------- merge without allocation */
 /* The same merge (and optional fused importance) as pa_merge_states, for callers that

@@ -23,7 +23,7 @@ import numpy as np
 __all__ = [
     "PA_F32", "PA_BF16", "PAError", "Context", "lib", "lib_path",
     "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head",
-    "pa_merge_states_noalloc", "EXPORTED", "select_fresh",
+    "pa_merge_states_noalloc", "pa_compose_states", "EXPORTED", "select_fresh",
 ]
 
 PA_F32, PA_BF16 = 0, 1
@@ -32,7 +32,7 @@ _ERRORS = {-1: "PA_EINVAL", -2: "PA_EALIGN", -3: "PA_EUNSUPPORTED", -4: "PA_ENOM
            -5: "PA_ECUDA", -6: "PA_ETIMEOUT"}
 EXPORTED = ("pa_init", "pa_destroy", "pa_last_error", "pa_sync_status", "pa_version",
             "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head",
-            "pa_merge_states_noalloc")
+            "pa_merge_states_noalloc", "pa_compose_states")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -63,7 +63,7 @@ class _MergeDesc(ctypes.Structure):
                 ("o_fresh", ctypes.c_void_p), ("lse_fresh", ctypes.c_void_p),
                 ("o_cached", ctypes.c_void_p), ("lse_cached", ctypes.c_void_p),
                 ("fresh", ctypes.c_void_p), ("o", ctypes.c_void_p), ("lse", ctypes.c_void_p),
-                ("w", ctypes.c_void_p)]
+                ("w", ctypes.c_void_p), ("cached_per_group", ctypes.c_int)]
 
 
 _LIB = None
@@ -90,8 +90,10 @@ def lib():
         L.pa_merge_states.argtypes = [vp, ctypes.POINTER(_MergeDesc), vp]
         L.pa_merge_states_noalloc.argtypes = [ctypes.POINTER(_MergeDesc), vp]
         L.pa_importance.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
+        L.pa_compose_states.argtypes = [vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
         L.pa_relayout_seq2head.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, vp]
         for f in ("pa_init", "pa_sync_status", "pa_partition_attn", "pa_merge_states", "pa_merge_states_noalloc",
+                  "pa_compose_states",
                   "pa_importance", "pa_relayout_seq2head"):
             getattr(L, f).restype = ci
         _LIB = L
@@ -179,9 +181,10 @@ def pa_partition_attn(ctx: Context, q, k, v, part_off, G, fresh, o_part, lse_par
 
 
 def pa_merge_states(ctx: Context, part_off, G, fresh, o_fresh, lse_fresh, o_cached, lse_cached,
-                    o, lse, w=None, stream=None):
+                    o, lse, w=None, stream=None, cached_per_group=False):
     """Merge fresh / cached states per the mask; o [B, H, N, D], lse [B, H, N]; w [QG, P]
-    (fused importance) optional."""
+    (fused importance) optional.  cached_per_group: the cache holds one composed state per
+    KV group ([KG, B, H, N, D], from pa_compose_states)."""
     P, B, H, N, D = o_fresh.shape
     off = _host_i32(part_off)
     fr = _host_u8(fresh)
@@ -190,8 +193,17 @@ def pa_merge_states(ctx: Context, part_off, G, fresh, o_fresh, lse_fresh, o_cach
                    None if o_cached is None else o_cached.data_ptr(),
                    None if lse_cached is None else lse_cached.data_ptr(),
                    None if fr is None else fr.ctypes.data, o.data_ptr(), lse.data_ptr(),
-                   None if w is None else w.data_ptr())
+                   None if w is None else w.data_ptr(), 1 if cached_per_group else 0)
     _check(ctx.ptr, lib().pa_merge_states(ctx.ptr, ctypes.byref(d), _stream(stream)))
+
+
+def pa_compose_states(ctx: Context, o_part, lse_part, factor, o_group, lse_group, stream=None):
+    """Compose every `factor` consecutive partitions' states into one (no recomputation):
+    o_part [P, B, H, N, D], lse_part [P, B, H, N] -> o_group [C, ...], lse_group [C, ...]."""
+    P, B, H, N, D = o_part.shape
+    _check(ctx.ptr, lib().pa_compose_states(ctx.ptr, _dtype_code(o_part), B, H, N, D, P, int(factor),
+                                            o_part.data_ptr(), lse_part.data_ptr(),
+                                            o_group.data_ptr(), lse_group.data_ptr(), _stream(stream)))
 
 
 def pa_merge_states_noalloc(part_off, G, fresh, o_fresh, lse_fresh, o_cached, lse_cached, o, lse,

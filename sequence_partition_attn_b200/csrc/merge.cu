@@ -80,6 +80,19 @@ __global__ void __launch_bounds__(kMR) merge_kernel(const __grid_constant__ Merg
   const size_t BHN = static_cast<size_t>(prm.BH) * prm.N;
   const size_t hrow0 = static_cast<size_t>(bh) * prm.N + r0;
 
+  // Where each partition's state comes from for this block's query group: e >= 0, fresh
+  // state e; e == -1, nothing (a partition of a reused group whose composed state sits in
+  // the group's first slot); e <= -2, cached state -e - 2 (partition p, or KV group p/G
+  // when the cache holds one composed state per group).
+  __shared__ int s_state[PA_MAX_P];
+  for (int p = threadIdx.x; p < P; p += kMR) {
+    int e = p;
+    if (!fresh_bit(prm.fresh_bits, qg, p))
+      e = prm.cached_per_group ? (p % prm.G == 0 ? -(p / prm.G) - 2 : -1) : -p - 2;
+    s_state[p] = e;
+  }
+  __syncthreads();
+
   // ---- phase 1: LSE and weights, one thread per row
   {
     const int t = threadIdx.x;
@@ -87,8 +100,10 @@ __global__ void __launch_bounds__(kMR) merge_kernel(const __grid_constant__ Merg
     float m = -INFINITY, l = 0.0f;
     if (ok) {
       for (int p = 0; p < P; ++p) {
-        const float* src = fresh_bit(prm.fresh_bits, qg, p) ? prm.lse_fresh : prm.lse_cached;
-        const float L = src[p * BHN + hrow0 + t];
+        const int e = s_state[p];
+        if (e == -1) continue;
+        const float* src = e >= 0 ? prm.lse_fresh : prm.lse_cached;
+        const float L = src[(e >= 0 ? e : -e - 2) * BHN + hrow0 + t];
         if (L > m) {
           l = l * expf(m - L) + 1.0f;
           m = L;
@@ -101,9 +116,10 @@ __global__ void __launch_bounds__(kMR) merge_kernel(const __grid_constant__ Merg
     if (ok) prm.lse[hrow0 + t] = lse;
     for (int p = 0; p < P; ++p) {
       float w = 0.0f;
-      if (ok && lse > -INFINITY) {
-        const float* src = fresh_bit(prm.fresh_bits, qg, p) ? prm.lse_fresh : prm.lse_cached;
-        w = expf(src[p * BHN + hrow0 + t] - lse);
+      const int e = s_state[p];
+      if (ok && lse > -INFINITY && e != -1) {
+        const float* src = e >= 0 ? prm.lse_fresh : prm.lse_cached;
+        w = expf(src[(e >= 0 ? e : -e - 2) * BHN + hrow0 + t] - lse);
       }
       sW[p * (kMR + 1) + t] = w;
     }
@@ -133,10 +149,11 @@ __global__ void __launch_bounds__(kMR) merge_kernel(const __grid_constant__ Merg
         const int p = p0 + u * SPW + slot;
         wt[u] = 0.0f;
         v[u] = make_uint4(0, 0, 0, 0);
-        if (p < P) {
+        const int e = p < P ? s_state[p] : -1;
+        if (e != -1) {
           wt[u] = sW[p * (kMR + 1) + i];
-          const uint8_t* base = fresh_bit(prm.fresh_bits, qg, p) ? of : oc;
-          v[u] = __ldg(reinterpret_cast<const uint4*>(base + p * BHN * kRowBytes + rowoff));
+          const uint8_t* base = e >= 0 ? of : oc;
+          v[u] = __ldg(reinterpret_cast<const uint4*>(base + (e >= 0 ? e : -e - 2) * BHN * kRowBytes + rowoff));
         }
       }
 #pragma unroll

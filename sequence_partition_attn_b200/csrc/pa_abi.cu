@@ -330,6 +330,10 @@ int pa_merge_states(pa_ctx* ctx, const pa_merge_desc* d, void* stream) {
   if (!d->o_fresh || !d->lse_fresh || !d->o || !d->lse) return fail(ctx, PA_EINVAL, "null tensor pointer");
   if (!all_fresh && (!d->o_cached || !d->lse_cached))
     return fail(ctx, PA_EINVAL, "cached states are NULL but the mask reuses some pairs");
+  if (d->cached_per_group != 0 && d->cached_per_group != 1)
+    return fail(ctx, PA_EINVAL, "cached_per_group=%d (0 or 1)", d->cached_per_group);
+  if (d->cached_per_group && d->w)
+    return fail(ctx, PA_EINVAL, "importance needs per-partition cached states (w must be NULL with cached_per_group)");
   if (!aligned(d->o_fresh, 16) || !aligned(d->o, 16) || (d->o_cached && !aligned(d->o_cached, 16)))
     return fail(ctx, PA_EALIGN, "o_fresh, o_cached and o must be 16-byte aligned");
   if (!aligned(d->lse_fresh, 4) || !aligned(d->lse, 4) || (d->lse_cached && !aligned(d->lse_cached, 4)) ||
@@ -360,12 +364,61 @@ int pa_merge_states(pa_ctx* ctx, const pa_merge_desc* d, void* stream) {
   prm.G = t.G;
   prm.QG = t.QG;
   prm.blocks_per_bh = bpb;
+  prm.cached_per_group = d->cached_per_group;
   memcpy(prm.part_off, t.part_off, sizeof prm.part_off);
   memcpy(prm.qg_row0, t.qg_row0, sizeof prm.qg_row0);
   memcpy(prm.fresh_bits, t.fresh_bits, sizeof prm.fresh_bits);
   int e = pa::launch_merge(prm, d->dtype, st);
   if (e) return cuda_fail(ctx, e, "merge launch");
   if (d->w) return launch_reduce(ctx, t, prm.blk_start, bpb, (int)BH, d->w, st);
+  return PA_OK;
+}
+
+int pa_compose_states(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int P, int factor,
+                      const void* o_part, const float* lse_part, void* o_group, float* lse_group,
+                      void* stream) {
+  if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
+  if (dtype != PA_BF16 && dtype != PA_F32) return fail(ctx, PA_EUNSUPPORTED, "dtype %d", (int)dtype);
+  if (D != 64 && D != 128) return fail(ctx, PA_EUNSUPPORTED, "D=%d (supported: 64, 128)", D);
+  if (B < 1 || H < 1 || N < 0) return fail(ctx, PA_EINVAL, "B=%d H=%d N=%d", B, H, N);
+  if (P < 1 || P > PA_MAX_P) return fail(ctx, PA_EINVAL, "P=%d outside [1, %d]", P, PA_MAX_P);
+  if (factor < 1 || factor > P) return fail(ctx, PA_EINVAL, "factor=%d outside [1, P=%d]", factor, P);
+  if (N == 0) return PA_OK;
+  if (!o_part || !lse_part || !o_group || !lse_group) return fail(ctx, PA_EINVAL, "null tensor pointer");
+  if (!aligned(o_part, 16) || !aligned(o_group, 16)) return fail(ctx, PA_EALIGN, "o_part and o_group must be 16-byte aligned");
+  if (!aligned(lse_part, 4) || !aligned(lse_group, 4)) return fail(ctx, PA_EALIGN, "lse arrays must be 4-byte aligned");
+  int rc = check_device(ctx);
+  if (rc) return rc;
+  const long long BH = static_cast<long long>(B) * H;
+  const size_t BHN = static_cast<size_t>(BH) * N;
+  const size_t row_bytes = static_cast<size_t>(D) * (dtype == PA_BF16 ? 2 : 4);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // One merge over each group's partitions: every row is one query group, all fresh.
+  for (int c = 0; c * factor < P; ++c) {
+    const int np = factor < P - c * factor ? factor : P - c * factor;
+    pa::MergeParams prm;
+    memset(&prm, 0, sizeof prm);
+    prm.o_fresh = static_cast<const uint8_t*>(o_part) + static_cast<size_t>(c) * factor * BHN * row_bytes;
+    prm.lse_fresh = lse_part + static_cast<size_t>(c) * factor * BHN;
+    prm.o = static_cast<uint8_t*>(o_group) + static_cast<size_t>(c) * BHN * row_bytes;
+    prm.lse = lse_group + static_cast<size_t>(c) * BHN;
+    prm.BH = (int)BH;
+    prm.N = N;
+    prm.D = D;
+    prm.P = np;
+    prm.G = np;
+    prm.QG = 1;
+    prm.qg_row0[0] = 0;
+    prm.qg_row0[1] = N;
+    for (int p = 0; p < np; ++p) prm.fresh_bits[0][p >> 5] |= 1u << (p & 31);
+    const int rpb = pa::merge_rows_per_block();
+    prm.blocks_per_bh = (N + rpb - 1) / rpb;
+    prm.blk_start[0] = 0;
+    prm.blk_start[1] = prm.blocks_per_bh;
+    if (BH * prm.blocks_per_bh > 0x7fffffffLL) return fail(ctx, PA_EINVAL, "too many row blocks");
+    int e = pa::launch_merge(prm, dtype, st);
+    if (e) return cuda_fail(ctx, e, "compose launch");
+  }
   return PA_OK;
 }
 
@@ -481,6 +534,10 @@ extern "C" int pa_merge_states_noalloc(const pa_merge_desc* d, void* stream) {
   if (!d->o_fresh || !d->lse_fresh || !d->o || !d->lse) return fail(nullptr, PA_EINVAL, "null tensor pointer");
   if (!all_fresh && (!d->o_cached || !d->lse_cached))
     return fail(nullptr, PA_EINVAL, "cached states are NULL but the mask reuses some pairs");
+  if (d->cached_per_group != 0 && d->cached_per_group != 1)
+    return fail(nullptr, PA_EINVAL, "cached_per_group=%d (0 or 1)", d->cached_per_group);
+  if (d->cached_per_group && d->w)
+    return fail(nullptr, PA_EINVAL, "importance needs per-partition cached states (w must be NULL with cached_per_group)");
   if (!aligned(d->o_fresh, 16) || !aligned(d->o, 16) || (d->o_cached && !aligned(d->o_cached, 16)))
     return fail(nullptr, PA_EALIGN, "o_fresh, o_cached and o must be 16-byte aligned");
   if (!aligned(d->lse_fresh, 4) || !aligned(d->lse, 4) || (d->lse_cached && !aligned(d->lse_cached, 4)) ||
@@ -519,6 +576,7 @@ extern "C" int pa_merge_states_noalloc(const pa_merge_desc* d, void* stream) {
   prm.G = t.G;
   prm.QG = t.QG;
   prm.blocks_per_bh = bpb;
+  prm.cached_per_group = d->cached_per_group;
   memcpy(prm.part_off, t.part_off, sizeof prm.part_off);
   memcpy(prm.qg_row0, t.qg_row0, sizeof prm.qg_row0);
   memcpy(prm.fresh_bits, t.fresh_bits, sizeof prm.fresh_bits);

@@ -53,6 +53,7 @@ struct MergeParams {
   float* lse;
   float* w_partial;               // [blocks][P] per-block importance sums, or null
   int BH, N, D, P, G, QG;
+  int cached_per_group;           // cached arrays hold one composed state per KV group
   int blocks_per_bh;              // row blocks per (b, h)
   int part_off[PA_MAX_P + 1];
   int qg_row0[PA_MAX_P + 1];

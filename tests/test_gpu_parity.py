@@ -251,3 +251,76 @@ def test_partition_state_reads_no_other_partition(pa, ctx):
     ctx.sync_status()
     assert torch.isfinite(o2[1].float()).all() and torch.isfinite(l2[1]).all()
     assert torch.equal(o1[1].view(torch.int16), o2[1].view(torch.int16)) and torch.equal(l1[1], l2[1])
+
+
+# --------------------------------------------------------------------------- group compose
+@pytest.mark.parametrize("dt,D,N,P,factor", [(torch.bfloat16, 128, 1500, 32, 4),
+                                              (torch.float32, 64, 700, 7, 3),
+                                              (torch.bfloat16, 64, 300, 5, 5)])
+def test_compose_states(pa, ctx, dt, D, N, P, factor):
+    off = W.part_offsets(N, P)
+    empty = [p for p in range(P) if off[p + 1] == off[p]]
+    o, l = _gen_states(7, P, 1, 2, N, D, dt, empty)
+    C = -(-P // factor)
+    og = torch.empty(C, 1, 2, N, D, dtype=dt, device=DEV)
+    lg = torch.empty(C, 1, 2, N, device=DEV)
+    pa.pa_compose_states(ctx, o.to(DEV), l.to(DEV), factor, og, lg)
+    ctx.sync_status()
+    ro, rl = O.compose_states(o.double().numpy(), l.double().numpy(), factor)
+    tol = TOL["bf16" if dt == torch.bfloat16 else "f32"]
+    assert maxerr(og.float().cpu().numpy(), ro) <= (tol["o"] if dt == torch.bfloat16 else 1e-5)
+    assert maxerr(lg.cpu().numpy(), rl) <= 1e-5 + 1e-6 * np.abs(rl[np.isfinite(rl)]).max()
+
+
+def test_merge_with_composed_cache_against_oracle(pa, ctx):
+    # seeded states (generated on the host) for both sides
+    N, P, G, D, H = 2900, 32, 4, 128, 2
+    off = W.part_offsets(N, P)
+    KG = P // G
+    fresh = (np.random.default_rng(3).random((KG, KG)) < 0.3).astype(np.uint8)
+    of, lf = _gen_states(11, P, 1, H, N, D, torch.bfloat16)
+    oc, lc = _gen_states(12, P, 1, H, N, D, torch.bfloat16)
+    ocg = torch.empty(KG, 1, H, N, D, dtype=torch.bfloat16, device=DEV)
+    lcg = torch.empty(KG, 1, H, N, device=DEV)
+    pa.pa_compose_states(ctx, oc.to(DEV), lc.to(DEV), G, ocg, lcg)
+    o = torch.empty(1, H, N, D, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(1, H, N, device=DEV)
+    pa.pa_merge_states(ctx, off, G, fresh, of.to(DEV), lf.to(DEV), ocg, lcg, o, lse, cached_per_group=True)
+    ctx.sync_status()
+    f64 = lambda x: x.double().numpy()   # noqa: E731
+    co, cl = O.compose_states(f64(oc), f64(lc), G)
+    ro, rl = O.merge_with_composed_cache(f64(of), f64(lf), co, cl, off, G, fresh)
+    # the composed cache is rounded to bf16 once more on the GPU side
+    assert maxerr(o.float().cpu().numpy(), ro) <= TOL["bf16"]["o"]
+    assert maxerr(lse.cpu().numpy(), rl) <= 1e-5 + 1e-6 * np.abs(rl).max()
+
+
+def test_merge_with_composed_cache(pa, ctx):
+    # 720p recipe on a reduced grid, states from the attention kernel: the composed-cache
+    # merge agrees with the per-partition merge (GPU against GPU: associativity).
+    wl = W.small_variant(W.workload(2), grid=(3, 45, 80), H=2)
+    t = W.make_qkv(wl)
+    kc, vc = W.make_cached_kv(wl, t["k"], t["v"])
+    off = W.part_offsets(wl.N, wl.P)
+    fresh = W.reuse_mask(wl)
+    q, k, v = (t[n].to(DEV) for n in ("q", "k", "v"))
+    P, B, H, N, D = wl.P, wl.B, wl.H, wl.N, wl.D
+    of = torch.zeros(P, B, H, N, D, dtype=torch.bfloat16, device=DEV)
+    lf = torch.zeros(P, B, H, N, device=DEV)
+    oc, lc = torch.zeros_like(of), torch.zeros_like(lf)
+    pa.pa_partition_attn(ctx, q, k, v, off, wl.G, fresh, of, lf)
+    pa.pa_partition_attn(ctx, q, kc.to(DEV), vc.to(DEV), off, wl.G, None, oc, lc)
+    ocg = torch.empty(wl.KG, B, H, N, D, dtype=torch.bfloat16, device=DEV)
+    lcg = torch.empty(wl.KG, B, H, N, device=DEV)
+    pa.pa_compose_states(ctx, oc, lc, wl.G, ocg, lcg)
+    o1 = torch.empty(B, H, N, D, dtype=torch.bfloat16, device=DEV)
+    l1 = torch.empty(B, H, N, device=DEV)
+    pa.pa_merge_states(ctx, off, wl.G, fresh, of, lf, ocg, lcg, o1, l1, cached_per_group=True)
+    o2, l2 = torch.empty_like(o1), torch.empty_like(l1)
+    pa.pa_merge_states(ctx, off, wl.G, fresh, of, lf, oc, lc, o2, l2)
+    ctx.sync_status()
+    assert maxerr(o1.float().cpu().numpy(), o2.float().cpu().numpy()) <= TOL["bf16"]["o"]
+    assert maxerr(l1.cpu().numpy(), l2.cpu().numpy()) <= 1e-5
+    w = torch.empty(wl.QG, P, device=DEV)
+    with pytest.raises(pa.PAError, match="PA_EINVAL"):
+        pa.pa_merge_states(ctx, off, wl.G, fresh, of, lf, ocg, lcg, o1, l1, w, cached_per_group=True)
