@@ -29,6 +29,13 @@ What is computed, and where the pages state it (DiTango web summary, Methodology
   Methodology 2 "Dynamic Group Compose"): cached states of consecutive partitions merge
   into one coarser state with no recomputation, and a reused KV group then contributes
   its single composed state to the merge.
+* state_drift / predict_fresh -- online error prediction between anchor steps (DiTango web
+  summary, Methodology 1 "Online Prediction": changes of the local states, which are
+  always computed, stand in for the drift of the reused remote ones).  state_drift sums,
+  per (query group, partition) over the selected pairs, |O_new - O_ref|^2 and |O_ref|^2
+  over batch, heads, rows and channels; predict_fresh recomputes a KV group when
+  w[qg][p] * sqrt(d2_own / r2_own) >= eps for some partition p of it, where the own
+  (diagonal) group's relative drift is the proxy.
 * relayout_seq2head -- the sequence-major -> head-major permutation that the Ulysses
   all-to-all performs, here on one device (SwiftFusion, Methodology 2).
 
@@ -46,7 +53,7 @@ import numpy as np
 __all__ = [
     "partition_states", "merge_states", "merge_with_reuse", "importance",
     "select_fresh", "relayout_seq2head", "group_bounds", "compose_states",
-    "merge_with_composed_cache",
+    "merge_with_composed_cache", "state_drift", "predict_fresh",
 ]
 
 
@@ -210,6 +217,45 @@ def select_fresh(w_stored, G, threshold):
     for g in range(QG):
         for kg in range(KG):
             m[g, kg] = 1 if np.any(w_stored[g, kg * G:(kg + 1) * G] >= threshold) else 0
+    return m
+
+
+def state_drift(o_new, o_ref, part_off, G, sel):
+    """(d2, r2), each [QG, P]: for every pair (query group qg, partition p) with
+    sel[qg, p // G], the sums over batch, heads, rows of qg and channels of
+    (o_new - o_ref)^2 and o_ref^2; 0 for other pairs.  o_new, o_ref: [P, B, H, N, D]."""
+    P = len(part_off) - 1
+    gb = group_bounds(part_off, G)
+    QG = len(gb) - 1
+    d2 = np.zeros((QG, P))
+    r2 = np.zeros((QG, P))
+    for qg in range(QG):
+        r0, r1 = int(gb[qg]), int(gb[qg + 1])
+        for p in range(P):
+            if not sel[qg, p // G]:
+                continue
+            a = o_new[p][:, :, r0:r1, :].astype(np.float64)
+            b = o_ref[p][:, :, r0:r1, :].astype(np.float64)
+            d2[qg, p] = ((a - b) ** 2).sum()
+            r2[qg, p] = (b ** 2).sum()
+    return d2, r2
+
+
+def predict_fresh(w_stored, d2, r2, G, eps):
+    """uint8[QG, KG]: recompute KV group kg for query group qg when some partition p of kg
+    has w_stored[qg, p] * drift[qg] >= eps, drift[qg] = sqrt(sum_p d2[qg, p] / sum_p r2[qg, p])
+    over the partitions of the own group kg = qg (0 when nothing was measured).  The own
+    group is always recomputed."""
+    QG, P = w_stored.shape
+    KG = -(-P // G)
+    m = np.zeros((QG, KG), dtype=np.uint8)
+    for qg in range(QG):
+        own = slice(qg * G, min((qg + 1) * G, P))
+        den = r2[qg, own].sum()
+        drift = np.sqrt(d2[qg, own].sum() / den) if den > 0 else 0.0
+        for kg in range(KG):
+            pred = max(w_stored[qg, p] * drift for p in range(kg * G, min((kg + 1) * G, P)))
+            m[qg, kg] = 1 if (kg == qg or pred >= eps) else 0
     return m
 
 

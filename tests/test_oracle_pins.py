@@ -463,3 +463,31 @@ def test_composed_state_is_attention_over_the_group():
     wide, wl, _ = O.partition_states(q, k, v, np.array([0, 20, 40]), 1, all_fresh(2), 0.5)
     np.testing.assert_allclose(co, wide, atol=1e-12)
     np.testing.assert_allclose(cl, wl, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- online prediction
+def test_state_drift_closed_forms():
+    rng = np.random.default_rng(30)
+    P, G, N, D = 4, 2, 20, 3
+    off = W.part_offsets(N, P)                   # 5 rows per partition, 2 query groups
+    ref = rng.standard_normal((P, 1, 2, N, D))
+    sel = np.array([[1, 0], [1, 1]], dtype=np.uint8)
+    d2, r2 = O.state_drift(ref, ref, off, G, sel)
+    assert not d2.any()
+    d2, r2 = O.state_drift(2 * ref, ref, off, G, sel)     # |2b - b|^2 = |b|^2
+    np.testing.assert_allclose(d2, r2, rtol=1e-14)
+    # brute force: query group 1 (rows 10..19), partition 1 (kv group 0, selected)
+    expect = sum(float(ref[1, 0, h, i, c]) ** 2 for h in range(2) for i in range(10, 20) for c in range(D))
+    assert abs(r2[1, 1] - expect) < 1e-10
+    assert r2[0, 2] == 0 and r2[0, 3] == 0                # query group 0 x kv group 1 not selected
+
+
+def test_predict_fresh_policy():
+    w = np.array([[0.6, 0.3, 0.07, 0.03], [0.1, 0.1, 0.5, 0.3]])
+    d2 = np.array([[4.0, 0.0, 0, 0], [0, 0, 1.0, 0.0]])
+    r2 = np.array([[100.0, 0.0, 0, 0], [0, 0, 25.0, 75.0]])   # drift: 0.2 and 0.1
+    m = O.predict_fresh(w, d2, r2, 2, eps=0.015)
+    # qg 0: kv group 1 max w = 0.07 -> 0.014 < 0.015 -> reuse; qg 1: kv group 0 0.1*0.1=0.01 -> reuse
+    np.testing.assert_array_equal(m, [[1, 0], [0, 1]])
+    m = O.predict_fresh(w, d2, r2, 2, eps=0.01)
+    np.testing.assert_array_equal(m, [[1, 1], [1, 1]])
