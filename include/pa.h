@@ -19,6 +19,12 @@
  *   pa_importance        partition importance w_p = exp(LSE_p - LSE), averaged per
  *                        (query group, partition) -- DiTango, Methodology 1 ("Error
  *                        modelling", "Anchor steps": importance refreshed at anchors).
+ *   pa_state_drift       per (query group, partition) sums of the squared change of the
+ *                        states between two steps and of the reference states' squares:
+ *                        the measurement behind the online prediction between anchor
+ *                        steps -- DiTango, Methodology 1 ("Online Prediction": the change
+ *                        of the always-computed local states stands in for the drift of
+ *                        the reused remote ones).
  *   pa_relayout_seq2head the sequence-major -> head-major permutation that the Ulysses
  *                        all-to-all performs, in sequence chunks -- SwiftFusion,
  *                        Methodology 2 ("Torus Attention": the all-to-all split into
@@ -198,6 +204,27 @@ int pa_merge_states_noalloc(const pa_merge_desc* desc, void* stream);
  * Errors: PA_EINVAL, PA_EALIGN, PA_ENOMEM, PA_ECUDA. */
 int pa_importance(pa_ctx* ctx, int B, int H, int N, int P, int G, const int32_t* part_off,
                   const float* lse_part, const float* lse, float* w, void* stream);
+
+/* ---------------------------------------------------------------- state drift */
+/* For every pair (query group qg, partition p) with sel[qg*KG + p/G] != 0:
+ *   d2[qg*P + p] = sum over b, h, rows i of qg and channels c of
+ *                  (o_new[p][b][h][i][c] - o_ref[p][b][h][i][c])^2,
+ *   r2[qg*P + p] = the same sum of o_ref[p][b][h][i][c]^2;
+ * 0 for the other pairs.  DiTango, Methodology 1, "Online Prediction": between anchor
+ * steps the change of the local states (own KV group, always recomputed) measured against
+ * the anchor's cached states estimates how fast the reused states drift; a caller turns
+ * d2 / r2 into a relative drift and combines it with the stored importance w.
+ *   o_new, o_ref  [P][B][H][N][D] device, dtype (the layout of pa_partition_attn's o_part);
+ *                 only the rows of selected pairs are read, so unselected pairs may hold
+ *                 anything.  D = 64 or 128.
+ *   sel           host uint8[QG*KG]; NULL selects every pair.
+ *   d2, r2        device float[QG*P], overwritten.  Sums are taken per 128-row block in
+ *                 fp32 and added over blocks in fp64 in a fixed order (deterministic).
+ * Uses the context's workspace (2 * P floats per 128-row block of each (b, h); same rule
+ * as pa_merge_states).  Errors: PA_EINVAL, PA_EALIGN, PA_EUNSUPPORTED, PA_ENOMEM, PA_ECUDA. */
+int pa_state_drift(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int P, int G,
+                   const int32_t* part_off, const uint8_t* sel, const void* o_new,
+                   const void* o_ref, float* d2, float* r2, void* stream);
 
 /* ---------------------------------------------------------------- relayout */
 /* dst[h][n][:] = src[n][h][:] for the tokens of sequence chunk `chunk` of `n_chunks`

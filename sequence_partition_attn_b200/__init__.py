@@ -8,7 +8,7 @@ names follow the C ABI in ``include/pa.h``:
 
     pa_init / Context            pa_partition_attn    pa_merge_states
     pa_importance                pa_relayout_seq2head pa_sync_status
-    pa_merge_states_noalloc
+    pa_merge_states_noalloc      pa_compose_states    pa_state_drift
 
 There is no fallback: if ``libpa.so`` is missing or the device is not sm_100 the calls
 raise.
@@ -23,7 +23,8 @@ import numpy as np
 __all__ = [
     "PA_F32", "PA_BF16", "PAError", "Context", "lib", "lib_path",
     "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head",
-    "pa_merge_states_noalloc", "pa_compose_states", "EXPORTED", "select_fresh",
+    "pa_merge_states_noalloc", "pa_compose_states", "pa_state_drift", "EXPORTED", "select_fresh",
+    "predict_fresh",
 ]
 
 PA_F32, PA_BF16 = 0, 1
@@ -32,7 +33,7 @@ _ERRORS = {-1: "PA_EINVAL", -2: "PA_EALIGN", -3: "PA_EUNSUPPORTED", -4: "PA_ENOM
            -5: "PA_ECUDA", -6: "PA_ETIMEOUT"}
 EXPORTED = ("pa_init", "pa_destroy", "pa_last_error", "pa_sync_status", "pa_version",
             "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head",
-            "pa_merge_states_noalloc", "pa_compose_states")
+            "pa_merge_states_noalloc", "pa_compose_states", "pa_state_drift")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -92,8 +93,9 @@ def lib():
         L.pa_importance.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
         L.pa_compose_states.argtypes = [vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
         L.pa_relayout_seq2head.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, vp]
+        L.pa_state_drift.argtypes = [vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp]
         for f in ("pa_init", "pa_sync_status", "pa_partition_attn", "pa_merge_states", "pa_merge_states_noalloc",
-                  "pa_compose_states",
+                  "pa_compose_states", "pa_state_drift",
                   "pa_importance", "pa_relayout_seq2head"):
             getattr(L, f).restype = ci
         _LIB = L
@@ -233,6 +235,19 @@ def pa_importance(ctx: Context, part_off, G, lse_part, lse, w, stream=None):
                                         _stream(stream)))
 
 
+def pa_state_drift(ctx: Context, part_off, G, sel, o_new, o_ref, d2, r2, stream=None):
+    """Per (query group, partition) sums of (o_new - o_ref)^2 and o_ref^2 over the pairs
+    selected by sel (uint8 [QG, KG] or None = all): o_new, o_ref [P, B, H, N, D];
+    d2, r2 [QG, P] f32, overwritten (0 for unselected pairs)."""
+    P, B, H, N, D = o_new.shape
+    off = _host_i32(part_off)
+    sl = _host_u8(sel)
+    _check(ctx.ptr, lib().pa_state_drift(ctx.ptr, _dtype_code(o_new), B, H, N, D, P, int(G),
+                                         off.ctypes.data, None if sl is None else sl.ctypes.data,
+                                         o_new.data_ptr(), o_ref.data_ptr(), d2.data_ptr(),
+                                         r2.data_ptr(), _stream(stream)))
+
+
 def pa_relayout_seq2head(ctx: Context, src, dst, n_chunks=1, chunk=-1, stream=None):
     """dst[h, n, :] = src[n, h, :] for sequence chunk `chunk` of `n_chunks` (-1 = all)."""
     N, H, D = src.shape
@@ -252,3 +267,28 @@ def select_fresh(w_stored, G: int, threshold: float) -> np.ndarray:
     pad = np.full((QG, KG * G), -np.inf)
     pad[:, :P] = w
     return (pad.reshape(QG, KG, G).max(axis=2) >= threshold).astype(np.uint8)
+
+
+def predict_fresh(w_stored, d2, r2, G: int, eps: float) -> np.ndarray:
+    """Host reuse selection between anchors from predicted error (DiTango web summary,
+    Methodology 1, "Error modelling" and "Online Prediction"): the error of reusing the
+    states of partition p for query group qg grows with its stored importance times the
+    drift of the states; the drift of the remote states is estimated by that of the own
+    KV group's states, which are recomputed every step:
+        drift[qg] = sqrt(sum_{p in own group} d2[qg, p] / sum_{p in own group} r2[qg, p]).
+    Returns uint8[QG, KG]: 1 (recompute) where max_{p in kg} w_stored[qg, p] * drift[qg]
+    reaches eps, and always on the diagonal (own group); d2, r2 as from pa_state_drift."""
+    w = np.asarray(w_stored, dtype=np.float64)
+    d2 = np.asarray(d2, dtype=np.float64)
+    r2 = np.asarray(r2, dtype=np.float64)
+    QG, P = w.shape
+    KG = -(-P // G)
+    own = (np.arange(P)[None, :] // G) == np.arange(QG)[:, None]
+    num = np.where(own, d2, 0.0).sum(axis=1)
+    den = np.where(own, r2, 0.0).sum(axis=1)
+    drift = np.sqrt(np.divide(num, den, out=np.zeros_like(num), where=den > 0))
+    pad = np.full((QG, KG * G), -np.inf)
+    pad[:, :P] = w * drift[:, None]
+    m = (pad.reshape(QG, KG, G).max(axis=2) >= eps).astype(np.uint8)
+    m[np.arange(QG), np.arange(QG)] = 1
+    return m

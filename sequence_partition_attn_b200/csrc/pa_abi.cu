@@ -458,6 +458,67 @@ int pa_importance(pa_ctx* ctx, int B, int H, int N, int P, int G, const int32_t*
   return launch_reduce(ctx, t, prm.blk_start, bpb, (int)BH, w, st);
 }
 
+int pa_state_drift(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int P, int G,
+                   const int32_t* part_off, const uint8_t* sel, const void* o_new, const void* o_ref,
+                   float* d2, float* r2, void* stream) {
+  if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
+  if (dtype != PA_BF16 && dtype != PA_F32) return fail(ctx, PA_EINVAL, "unknown dtype %d", (int)dtype);
+  if (B < 1 || H < 1 || N < 0) return fail(ctx, PA_EINVAL, "B=%d H=%d N=%d", B, H, N);
+  if (D != 64 && D != 128) return fail(ctx, PA_EUNSUPPORTED, "D=%d (64 or 128 supported)", D);
+  pa::AttnTables t;
+  int rc = build_tables(ctx, N, P, G, part_off, nullptr, t);
+  if (rc) return rc;
+  if (!d2 || !r2) return fail(ctx, PA_EINVAL, "d2 or r2 is NULL");
+  if (N > 0 && (!o_new || !o_ref)) return fail(ctx, PA_EINVAL, "null tensor pointer");
+  if (!aligned(o_new, 16) || !aligned(o_ref, 16) || !aligned(d2, 4) || !aligned(r2, 4))
+    return fail(ctx, PA_EALIGN, "o_new and o_ref must be 16-byte aligned, d2 and r2 4-byte aligned");
+  if ((rc = check_device(ctx))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH > 0x7fffffffLL) return fail(ctx, PA_EINVAL, "B*H too large");
+  pa::DriftParams prm;
+  memset(&prm, 0, sizeof prm);
+  const int rpb = pa::drift_rows_per_block();
+  int bpb = 0;
+  for (int qg = 0; qg < t.QG; ++qg) {
+    prm.blk_start[qg] = bpb;
+    bpb += (t.qg_row0[qg + 1] - t.qg_row0[qg] + rpb - 1) / rpb;
+  }
+  prm.blk_start[t.QG] = bpb;
+  const long long blocks = BH * bpb;
+  if (blocks > 0x7fffffffLL) return fail(ctx, PA_EINVAL, "too many row blocks");
+  if (blocks > 0) {
+    if ((rc = ensure_ws(ctx, static_cast<size_t>(blocks) * 2 * t.P * sizeof(float)))) return rc;
+    prm.o_new = o_new;
+    prm.o_ref = o_ref;
+    prm.partial = static_cast<float*>(ctx->ws);
+    prm.BH = (int)BH;
+    prm.N = N;
+    prm.P = t.P;
+    prm.G = t.G;
+    prm.QG = t.QG;
+    prm.blocks_per_bh = bpb;
+    memcpy(prm.qg_row0, t.qg_row0, sizeof prm.qg_row0);
+    for (int qg = 0; qg < t.QG; ++qg)
+      for (int kg = 0; kg < t.QG; ++kg)
+        if (!sel || sel[qg * t.QG + kg]) prm.sel_bits[qg][kg >> 5] |= 1u << (kg & 31);
+    int e = pa::launch_drift(prm, dtype, D, st);
+    if (e) return cuda_fail(ctx, e, "drift launch");
+  }
+  pa::ReducePairParams r;
+  memset(&r, 0, sizeof r);
+  r.partial = static_cast<const float*>(ctx->ws);
+  r.d2 = d2;
+  r.r2 = r2;
+  r.BH = (int)BH;
+  r.P = t.P;
+  r.QG = t.QG;
+  r.blocks_per_bh = bpb;
+  memcpy(r.blk_start, prm.blk_start, sizeof r.blk_start);
+  int e = pa::launch_reduce_pair(r, st);
+  return e ? cuda_fail(ctx, e, "drift reduce launch") : PA_OK;
+}
+
 int pa_relayout_seq2head(pa_ctx* ctx, const void* src, void* dst, int N, int H, int D, int elem_bytes,
                          int n_chunks, int chunk, void* stream) {
   if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");

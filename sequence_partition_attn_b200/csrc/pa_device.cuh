@@ -301,3 +301,24 @@ __device__ __forceinline__ float fast_log2(float x) {
   return y;
 }
 }  // namespace pa
+
+namespace pa {
+struct DriftParams {
+  const void* o_new;              // [P][B][H][N][D]
+  const void* o_ref;              // [P][B][H][N][D]
+  float* partial;                 // [blocks][2][P]: sums of (new - ref)^2, ref^2
+  int BH, N, P, G, QG;
+  int blocks_per_bh;
+  int qg_row0[PA_MAX_P + 1];
+  int blk_start[PA_MAX_P + 1];
+  uint32_t sel_bits[PA_MAX_P][PA_MAX_P / 32];
+};
+
+struct ReducePairParams {
+  const float* partial;           // [BH * blocks_per_bh][2][P]
+  float* d2;                      // [QG][P]
+  float* r2;                      // [QG][P]
+  int BH, P, QG, blocks_per_bh;
+  int blk_start[PA_MAX_P + 1];
+};
+}  // namespace pa

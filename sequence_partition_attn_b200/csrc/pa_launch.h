@@ -19,6 +19,10 @@ int merge_rows_per_block();
 int launch_importance(const ImportanceParams& prm, cudaStream_t st);
 int launch_reduce_w(const ReduceWParams& prm, cudaStream_t st);
 
+int drift_rows_per_block();
+int launch_drift(const DriftParams& prm, int dtype, int D, cudaStream_t st);
+int launch_reduce_pair(const ReducePairParams& prm, cudaStream_t st);
+
 int launch_relayout(const void* src, void* dst, long long n0, long long n1, int N, int H,
                     int row_bytes, int sm_count, cudaStream_t st);
 

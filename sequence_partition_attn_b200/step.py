@@ -4,8 +4,10 @@ A step takes Q, K, V of one denoising step already in HBM, computes the attentio
 the fresh (query group, KV group) pairs, and merges them with the cached states of the
 other pairs into (O, LSE) plus the partition importance w (DiTango web summary,
 Methodology 1-2).  ``Trajectory`` adds the host side of the selection: all pairs fresh at
-anchor steps (importance stored, cache refreshed), otherwise pairs whose stored
-importance falls below a threshold reuse the anchor's states.
+anchor steps (importance stored, cache refreshed); otherwise either pairs whose stored
+importance falls below a threshold reuse the anchor's states, or (online prediction) the
+own groups are computed first, their drift from the anchor measured, and pairs whose
+predicted error (importance times drift) stays below a bound reuse the anchor's states.
 
 Only orchestration lives here; every arithmetic step runs in libpa's kernels.
 """
@@ -15,7 +17,7 @@ import numpy as np
 import torch
 
 from . import (Context, pa_merge_states, pa_partition_attn, pa_relayout_seq2head,
-               select_fresh)
+               pa_state_drift, predict_fresh, select_fresh)
 
 
 def attn_flops(part_off, G: int, fresh, B: int, H: int, D: int) -> float:
@@ -89,16 +91,30 @@ class Trajectory:
     """Denoising trajectory with anchor steps and importance-driven reuse (host selection).
 
     At an anchor step every pair is fresh, the states become the cache and the importance
-    w is stored (copied to the host: QG*P floats, the only device-to-host transfer).  At
-    any other step the mask is ``select_fresh(w_stored, G, threshold)``; fresh pairs are
-    recomputed from the current K, V and merged with the anchor's cached states.
+    w is stored (copied to the host: QG*P floats).  Between anchors the mask comes from
+    one of two policies (DiTango web summary, Methodology 1):
+
+    * ``"threshold"``: ``select_fresh(w_stored, G, threshold)`` -- recompute where the
+      stored importance reaches the threshold.  No device-to-host transfer.
+    * ``"predict"`` (online prediction): the own (query group, KV group) pairs -- always
+      recomputed -- run first; ``pa_state_drift`` measures their states' change from the
+      anchor's cached states; ``predict_fresh(w_stored, d2, r2, G, threshold)`` recomputes
+      the pairs whose importance times that drift reaches the threshold (an error bound
+      here).  The other selected pairs then run in a second attention launch.  Costs one
+      2*QG*P-float device-to-host copy per step.
+
+    Fresh pairs are recomputed from the current K, V and merged with the anchor's cached
+    states.
     """
 
     def __init__(self, ctx, B, H, N, D, part_off, G, anchors, threshold, dtype=torch.bfloat16,
-                 device="cuda:0"):
+                 device="cuda:0", policy="threshold"):
+        if policy not in ("threshold", "predict"):
+            raise ValueError(f"unknown policy {policy!r}")
         self.ctx = ctx
         self.anchors = set(anchors)
         self.threshold = threshold
+        self.policy = policy
         self.G = G
         self.part_off = np.asarray(part_off, dtype=np.int32)
         P = len(self.part_off) - 1
@@ -111,7 +127,32 @@ class Trajectory:
         self.o = torch.empty(B, H, N, D, dtype=dtype, device=dev)
         self.lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
         self.w = torch.empty(self.QG, P, dtype=torch.float32, device=dev)
+        self.d2 = torch.empty(self.QG, P, dtype=torch.float32, device=dev)
+        self.r2 = torch.empty_like(self.d2)
         self.w_stored = None
+        self.drift = None                   # (d2, r2) host copies of the last prediction
+
+    def _mask(self, q, k, v, stream):
+        if self.policy == "threshold":
+            mask = select_fresh(self.w_stored, self.G, self.threshold)
+            pa_partition_attn(self.ctx, q, k, v, self.part_off, self.G, mask, self.o_fresh,
+                              self.lse_fresh, stream=stream)
+            return mask
+        own = np.eye(self.QG, dtype=np.uint8)
+        pa_partition_attn(self.ctx, q, k, v, self.part_off, self.G, own, self.o_fresh,
+                          self.lse_fresh, stream=stream)
+        pa_state_drift(self.ctx, self.part_off, self.G, own, self.o_fresh, self.cache_o,
+                       self.d2, self.r2, stream=stream)
+        self.ctx.sync_status(stream)
+        d2 = self.d2.cpu().numpy().astype(np.float64)
+        r2 = self.r2.cpu().numpy().astype(np.float64)
+        self.drift = (d2, r2)
+        mask = predict_fresh(self.w_stored, d2, r2, self.G, self.threshold)
+        rest = mask & ~own.astype(bool)
+        if rest.any():
+            pa_partition_attn(self.ctx, q, k, v, self.part_off, self.G, rest, self.o_fresh,
+                              self.lse_fresh, stream=stream)
+        return mask
 
     def step(self, s: int, q, k, v, stream=None) -> np.ndarray:
         """Run step s on device tensors q, k, v; returns the mask it used (uint8[QG, KG])."""
@@ -123,9 +164,7 @@ class Trajectory:
                             None, None, self.o, self.lse, self.w, stream=stream)
             self.w_stored = self.w.cpu().numpy().astype(np.float64)
             return mask
-        mask = select_fresh(self.w_stored, self.G, self.threshold)
-        pa_partition_attn(self.ctx, q, k, v, self.part_off, self.G, mask, self.o_fresh,
-                          self.lse_fresh, stream=stream)
+        mask = self._mask(q, k, v, stream)
         pa_merge_states(self.ctx, self.part_off, self.G, mask, self.o_fresh, self.lse_fresh,
                         self.cache_o, self.cache_lse, self.o, self.lse, self.w, stream=stream)
         return mask

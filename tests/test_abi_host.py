@@ -78,3 +78,18 @@ def test_host_reuse_selection_matches_the_oracle(seed):
     w = rng.dirichlet(np.ones(P), size=QG) * rng.uniform(0.2, 1.5)
     w[rng.random(w.shape) < 0.2] = 0.05                 # exact threshold hits
     np.testing.assert_array_equal(pa.select_fresh(w, G, 0.05), O.select_fresh(w, G, 0.05))
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_host_error_prediction_matches_the_oracle(seed):
+    rng = np.random.default_rng(100 + seed)
+    P = int(rng.integers(1, 33))
+    G = int(rng.integers(1, P + 1))
+    QG = -(-P // G)
+    w = rng.dirichlet(np.ones(P), size=QG)
+    d2 = rng.uniform(0, 0.01, size=(QG, P)) * (rng.random((QG, P)) < 0.8)
+    r2 = rng.uniform(0.5, 2.0, size=(QG, P))
+    r2[rng.random(QG) < 0.2] = 0.0                      # groups with nothing measured
+    eps = float(np.quantile(w, 0.5)) * 0.05
+    np.testing.assert_array_equal(pa.predict_fresh(w, d2, r2, G, eps),
+                                  O.predict_fresh(w, d2, r2, G, eps))

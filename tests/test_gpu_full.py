@@ -101,13 +101,16 @@ def test_720p_step_full_size_sampled_rows(pa):
     ctx.close()
 
 
-def _run_trajectory(pa, wl, quality_heads=0):
+def _run_trajectory(pa, wl, quality_heads=0, policy="threshold", margin=0.15):
     from sequence_partition_attn_b200.step import Trajectory
     off = W.part_offsets(wl.N, wl.P)
     host = W.make_qkv(wl)
     q, k, v = host["q"], host["k"], host["v"]
     ctx = pa.Context(0)
-    traj = Trajectory(ctx, wl.B, wl.H, wl.N, wl.D, off, wl.G, wl.anchors, wl.threshold, device=DEV)
+    traj = Trajectory(ctx, wl.B, wl.H, wl.N, wl.D, off, wl.G, wl.anchors, wl.threshold, device=DEV,
+                      policy=policy)
+    own = np.eye(wl.QG, dtype=np.uint8)
+    ref_w = None
     qd = q.to(DEV)
     qf = W.to_f64(q)
     ones = np.ones((wl.QG, wl.KG), dtype=np.uint8)
@@ -129,12 +132,25 @@ def _run_trajectory(pa, wl, quality_heads=0):
             ref_cache = (of, lf)
             ro, rl = O.merge_states(list(of), list(lf))
             rw = O.importance(lf, rl, off, wl.G)
+            ref_w = rw
             assert maxerr(traj.w_stored, rw) <= tol["w"]
             # pairs the oracle's own w would select differently at the threshold
             flips = int((O.select_fresh(rw, wl.G, wl.threshold) !=
                          O.select_fresh(traj.w_stored, wl.G, wl.threshold)).sum())
         else:
             ro, rl, _ = O.merge_with_reuse(of, lf, ref_cache[0], ref_cache[1], off, wl.G, mask)
+            if policy == "predict":
+                # the oracle's own prediction from its own-group states, anchor cache and w;
+                # pairs whose predicted error lies within `margin` of the bound may differ
+                # (bf16 states on the GPU), every other pair must agree
+                d2, r2 = O.state_drift(of, ref_cache[0], off, wl.G, own)
+                rmask = O.predict_fresh(ref_w, d2, r2, wl.G, wl.threshold)
+                drift = np.sqrt(np.diag(d2.reshape(wl.QG, wl.KG, wl.G).sum(2)) /
+                                np.diag(r2.reshape(wl.QG, wl.KG, wl.G).sum(2)))
+                pred = (ref_w * drift[:, None]).reshape(wl.QG, wl.KG, wl.G).max(2)
+                firm = (np.abs(pred / wl.threshold - 1.0) > margin) | own.astype(bool)
+                assert (mask[firm] == rmask[firm]).all(), (s, mask, rmask)
+                flips = int((mask != rmask).sum())
         err_o, err_l = maxerr(o, ro), maxerr(lse, rl)
         assert err_o <= tol["o"] and err_l <= tol["lse"], (s, err_o, err_l)
         q_err = float("nan")
@@ -165,6 +181,22 @@ def test_denoising_trajectory_with_reuse(pa):
     report = _run_trajectory(pa, wl, quality_heads=4)
     assert report[0][1] == wl.QG * wl.KG and report[5][1] == wl.QG * wl.KG
     assert any(r[1] < wl.QG * wl.KG for r in report)           # reuse happened
+
+
+def test_denoising_trajectory_online_prediction(pa):
+    # same shape and drift; between anchors the mask comes from the online prediction
+    # (own groups first, their drift from the anchor times the stored importance against
+    # an error bound of 1e-3: with these inputs the oracle recomputes 8, 10, 29, 57 of the
+    # 64 pairs on the four steps after each anchor -- own groups only on the first, more as
+    # the drift grows)
+    base = W.workload(3)
+    wl = W.small_variant(base, grid=base.grid, H=base.H, threshold=1e-3)
+    report = _run_trajectory(pa, wl, quality_heads=4, policy="predict")
+    fresh = [r[1] for r in report]
+    assert fresh[0] == wl.QG * wl.KG and fresh[5] == wl.QG * wl.KG
+    assert fresh[1] == wl.QG and fresh[6] == wl.QG             # own groups only
+    assert fresh[4] > fresh[2] and fresh[9] > fresh[7]          # more recomputed as drift grows
+    assert fresh[4] < wl.QG * wl.KG
 
 
 def test_ulysses_layout_full_size(pa):

@@ -324,3 +324,59 @@ def test_merge_with_composed_cache(pa, ctx):
     w = torch.empty(wl.QG, P, device=DEV)
     with pytest.raises(pa.PAError, match="PA_EINVAL"):
         pa.pa_merge_states(ctx, off, wl.G, fresh, of, lf, ocg, lcg, o1, l1, w, cached_per_group=True)
+
+
+# --------------------------------------------------------------------------- state drift
+@pytest.mark.parametrize("dt,D,N,P,G,B,H,sel_kind", [
+    (torch.bfloat16, 128, 2900, 32, 4, 1, 2, "random"),
+    (torch.float32, 64, 517, 5, 2, 2, 2, "all"),
+    (torch.bfloat16, 64, 16, 5, 1, 1, 3, "own"),        # an empty partition, 4-row groups
+    (torch.bfloat16, 128, 4096, 8, 1, 1, 4, "own"),     # trajectory shape, fewer heads
+])
+def test_state_drift_against_oracle(pa, ctx, dt, D, N, P, G, B, H, sel_kind):
+    off = W.part_offsets(N, P)
+    QG = -(-P // G)
+    empty = [p for p in range(P) if off[p + 1] == off[p]]
+    o_new, _ = _gen_states(21, P, B, H, N, D, dt, empty)
+    o_ref, _ = _gen_states(22, P, B, H, N, D, dt, empty)
+    if sel_kind == "random":
+        sel = (np.random.default_rng(5).random((QG, QG)) < 0.4).astype(np.uint8)
+        np.fill_diagonal(sel, 1)
+    elif sel_kind == "own":
+        sel = np.eye(QG, dtype=np.uint8)
+    else:
+        sel = np.ones((QG, QG), dtype=np.uint8)
+    o_new_d = o_new.to(DEV)
+    # states of unselected pairs may hold anything: poison every row outside the selection
+    gb = W.group_row_bounds(off, G)
+    for qg in range(QG):
+        for p in range(P):
+            if not sel[qg, p // G]:
+                o_new_d[p, :, :, gb[qg]:gb[qg + 1]] = float("nan")
+    d2 = torch.full((QG, P), -1.0, device=DEV)
+    r2 = torch.full((QG, P), -1.0, device=DEV)
+    pa.pa_state_drift(ctx, off, G, None if sel_kind == "all" else sel, o_new_d, o_ref.to(DEV), d2, r2)
+    ctx.sync_status()
+    rd, rr = O.state_drift(o_new.double().numpy(), o_ref.double().numpy(), off, G, sel)
+    gd, gr = d2.cpu().numpy().astype(np.float64), r2.cpu().numpy().astype(np.float64)
+    assert np.isfinite(gd).all() and np.isfinite(gr).all()
+    assert np.abs(gd - rd).max() <= 1e-5 * max(rd.max(), 1.0)
+    assert np.abs(gr - rr).max() <= 1e-5 * max(rr.max(), 1.0)
+    assert (gd[rd == 0] == 0).all() and (gr[rr == 0] == 0).all()
+
+
+def test_state_drift_empty_sequence_and_errors(pa, ctx):
+    P, G = 4, 2
+    off = np.zeros(P + 1, dtype=np.int32)
+    o = torch.empty(P, 1, 1, 0, 64, dtype=torch.bfloat16, device=DEV)
+    d2 = torch.full((2, P), 7.0, device=DEV)
+    r2 = torch.full((2, P), 7.0, device=DEV)
+    pa.pa_state_drift(ctx, off, G, None, o, o, d2, r2)
+    ctx.sync_status()
+    assert (d2.cpu() == 0).all() and (r2.cpu() == 0).all()
+    o = torch.zeros(P, 1, 1, 64, 96, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(pa.PAError, match="PA_EUNSUPPORTED"):
+        pa.pa_state_drift(ctx, W.part_offsets(64, P), G, None, o, o, d2, r2)
+    o = torch.zeros(P, 1, 1, 64, 64, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(pa.PAError, match="PA_EINVAL"):
+        pa.pa_state_drift(ctx, W.part_offsets(63, P), G, None, o, o, d2, r2)
