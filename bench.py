@@ -369,6 +369,24 @@ def run_ours(args, ws, rank, local):
                                             "cache_bytes_before": float(B * H * N) * row_b * wl.P,
                                             "cache_bytes_after": float(B * H * N) * row_b * KG}}
         del ocg, lcg
+        # ---- online prediction: drift of the own groups' states from the cached states
+        own = np.eye(wl.QG, dtype=np.uint8)
+        d2 = torch.empty(wl.QG, wl.P, dtype=torch.float32, device=dev)
+        r2 = torch.empty_like(d2)
+        for _ in range(3):
+            pa.pa_state_drift(ctx, off, G, own, step.o_fresh, step.o_cached, d2, r2)
+        m0.record(stream)
+        for _ in range(reps):
+            pa.pa_state_drift(ctx, off, G, own, step.o_fresh, step.o_cached, d2, r2)
+        m1.record(stream)
+        torch.cuda.synchronize()
+        ctx.sync_status()
+        dr_ms = m0.elapsed_time(m1) / reps
+        own_rows = sum(int(gb[qg + 1] - gb[qg]) * min(G, wl.P - qg * G) for qg in range(wl.QG))
+        dr_bytes = 2.0 * B * H * own_rows * D * 2
+        composed_extra["state_drift"] = {"ms": dr_ms, "gbs": dr_bytes / (dr_ms / 1e3) / 1e9,
+                                         "bytes": dr_bytes, "selection": "own groups"}
+        del d2, r2
     else:
         composed_extra = {}
     del step
