@@ -8,8 +8,10 @@
 //   r2[qg][p] = the same sum of O_ref^2.
 // Bound by HBM reads of the two state sets.  A block owns up to 128 rows of one query group
 // of one (b, h); the rows of a partition's states are contiguous, so the block reads
-// nrows * D * elem bytes per selected partition with 16-byte coalesced loads.  Per-block
-// sums go to a workspace and are added per query group in a fixed order (deterministic).
+// nrows * D * elem bytes per selected partition with 16-byte coalesced loads, 8 per
+// tensor in flight per thread.  Warps keep per-partition sums in shared memory and the
+// block adds them once at the end; per-block sums go to a workspace and are added per
+// query group in a fixed order (deterministic).
 #include "pa_device.cuh"
 #include "pa_launch.h"
 
@@ -18,6 +20,7 @@ namespace {
 
 constexpr int kRows = 128;
 constexpr int kThreads = 256;
+constexpr int kBatch = 8;
 
 template <typename T> struct Elems;
 template <> struct Elems<float> {
@@ -50,7 +53,10 @@ template <> struct Elems<__nv_bfloat16> {
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) drift_kernel(const __grid_constant__ DriftParams prm) {
   constexpr int kChunks = D * sizeof(T) / 16;      // 16-byte pieces per state row
-  __shared__ float s_red[2][kThreads / 32];
+  constexpr int kWarps = kThreads / 32;
+  // Per-warp sums of every partition; the block adds them once at the end, so warps run
+  // ahead from one partition to the next without a block barrier in between.
+  __shared__ float s_red[2][PA_MAX_P][kWarps];
   const int bh = blockIdx.x / prm.blocks_per_bh;
   const int blk = blockIdx.x - bh * prm.blocks_per_bh;
   int qg = 0;
@@ -62,55 +68,86 @@ __global__ void __launch_bounds__(kThreads) drift_kernel(const __grid_constant__
   const uint4* a = static_cast<const uint4*>(prm.o_new);
   const uint4* b = static_cast<const uint4*>(prm.o_ref);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* out = prm.partial + static_cast<size_t>(blockIdx.x) * 2 * prm.P;
+  const int n = nrows * kChunks;
   for (int p = 0; p < prm.P; ++p) {
-    if (!fresh_bit(prm.sel_bits, qg, p / prm.G)) {
-      if (threadIdx.x == 0) {
-        out[p] = 0.0f;
-        out[prm.P + p] = 0.0f;
-      }
-      continue;
-    }
-    const size_t base = (static_cast<size_t>(p) * BHN + first) * kChunks;
     float dd = 0.0f, rr = 0.0f;
-    for (int idx = threadIdx.x; idx < nrows * kChunks; idx += kThreads)
-      Elems<T>::acc(__ldg(a + base + idx), __ldg(b + base + idx), dd, rr);
+    if (fresh_bit(prm.sel_bits, qg, p / prm.G)) {
+      const size_t base = (static_cast<size_t>(p) * BHN + first) * kChunks;
+      // kBatch chunks of each tensor in flight per thread.
+      for (int i0 = 0; i0 < n; i0 += kBatch * kThreads) {
+        uint4 va[kBatch], vb[kBatch];
+        if (i0 + kBatch * kThreads <= n) {          // whole batch in range: unguarded loads
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      dd += __shfl_xor_sync(0xffffffffu, dd, off);
-      rr += __shfl_xor_sync(0xffffffffu, rr, off);
+          for (int k = 0; k < kBatch; ++k) {
+            va[k] = __ldg(a + base + i0 + threadIdx.x + k * kThreads);
+            vb[k] = __ldg(b + base + i0 + threadIdx.x + k * kThreads);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < kBatch; ++k) {
+            const int idx = i0 + threadIdx.x + k * kThreads;
+            va[k] = idx < n ? __ldg(a + base + idx) : make_uint4(0, 0, 0, 0);
+            vb[k] = idx < n ? __ldg(b + base + idx) : make_uint4(0, 0, 0, 0);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) Elems<T>::acc(va[k], vb[k], dd, rr);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        dd += __shfl_xor_sync(0xffffffffu, dd, off);
+        rr += __shfl_xor_sync(0xffffffffu, rr, off);
+      }
     }
     if (lane == 0) {
-      s_red[0][warp] = dd;
-      s_red[1][warp] = rr;
+      s_red[0][p][warp] = dd;
+      s_red[1][p][warp] = rr;
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float sd = 0.0f, sr = 0.0f;
-      for (int w = 0; w < kThreads / 32; ++w) {
-        sd += s_red[0][w];
-        sr += s_red[1][w];
-      }
-      out[p] = sd;
-      out[prm.P + p] = sr;
+  }
+  __syncthreads();
+  float* out = prm.partial + static_cast<size_t>(blockIdx.x) * 2 * prm.P;
+  for (int p = threadIdx.x; p < prm.P; p += kThreads) {
+    float sd = 0.0f, sr = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      sd += s_red[0][p][w];
+      sr += s_red[1][p][w];
     }
-    __syncthreads();
+    out[p] = sd;
+    out[prm.P + p] = sr;
   }
 }
 
-__global__ void __launch_bounds__(128) reduce_pair_kernel(const __grid_constant__ ReducePairParams prm) {
-  const int qg = blockIdx.x;
-  const int b0 = prm.blk_start[qg], b1 = prm.blk_start[qg + 1];
-  for (int p = threadIdx.x; p < prm.P; p += blockDim.x) {
-    double sd = 0.0, sr = 0.0;
-    for (int bh = 0; bh < prm.BH; ++bh)
-      for (int b = b0; b < b1; ++b) {
-        const float* part = prm.partial + (static_cast<size_t>(bh) * prm.blocks_per_bh + b) * 2 * prm.P;
-        sd += part[p];
-        sr += part[prm.P + p];
-      }
-    prm.d2[qg * prm.P + p] = static_cast<float>(sd);
-    prm.r2[qg * prm.P + p] = static_cast<float>(sr);
+// One block per (query group, partition): fixed assignment of the (b*h, row block)
+// partial sums to threads, fp64 sums, fixed-shape tree (deterministic).
+constexpr int kRT = 256;
+
+__global__ void __launch_bounds__(kRT) reduce_pair_kernel(const __grid_constant__ ReducePairParams prm) {
+  __shared__ double s_sum[2][kRT];
+  const int qg = blockIdx.x / prm.P, p = blockIdx.x - qg * prm.P;
+  const int b0 = prm.blk_start[qg], nb = prm.blk_start[qg + 1] - b0;
+  const long long E = static_cast<long long>(prm.BH) * nb;
+  double sd = 0.0, sr = 0.0;
+  for (long long e = threadIdx.x; e < E; e += kRT) {
+    const long long bh = e / nb;
+    const long long b = e - bh * nb;
+    const float* part = prm.partial + (bh * prm.blocks_per_bh + b0 + b) * 2 * prm.P;
+    sd += part[p];
+    sr += part[prm.P + p];
+  }
+  s_sum[0][threadIdx.x] = sd;
+  s_sum[1][threadIdx.x] = sr;
+  __syncthreads();
+  for (int off = kRT / 2; off > 0; off >>= 1) {
+    if (static_cast<int>(threadIdx.x) < off) {
+      s_sum[0][threadIdx.x] += s_sum[0][threadIdx.x + off];
+      s_sum[1][threadIdx.x] += s_sum[1][threadIdx.x + off];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    prm.d2[qg * prm.P + p] = static_cast<float>(s_sum[0][0]);
+    prm.r2[qg * prm.P + p] = static_cast<float>(s_sum[1][0]);
   }
 }
 
@@ -131,7 +168,7 @@ int launch_drift(const DriftParams& prm, int dtype, int D, cudaStream_t st) {
 }
 
 int launch_reduce_pair(const ReducePairParams& prm, cudaStream_t st) {
-  reduce_pair_kernel<<<prm.QG, 128, 0, st>>>(prm);
+  reduce_pair_kernel<<<prm.QG * prm.P, kRT, 0, st>>>(prm);
   return static_cast<int>(cudaGetLastError());
 }
 

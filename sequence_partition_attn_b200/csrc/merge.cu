@@ -85,6 +85,8 @@ __global__ void __launch_bounds__(kMR) merge_kernel(const __grid_constant__ Merg
   // the group's first slot); e <= -2, cached state -e - 2 (partition p, or KV group p/G
   // when the cache holds one composed state per group).
   __shared__ int s_state[PA_MAX_P];
+  __shared__ int s_act[PA_MAX_P];                  // partitions with a state, in order
+  __shared__ int s_nact;
   for (int p = threadIdx.x; p < P; p += kMR) {
     int e = p;
     if (!fresh_bit(prm.fresh_bits, qg, p))
@@ -92,6 +94,14 @@ __global__ void __launch_bounds__(kMR) merge_kernel(const __grid_constant__ Merg
     s_state[p] = e;
   }
   __syncthreads();
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int p = 0; p < P; ++p)
+      if (s_state[p] != -1) s_act[n++] = p;
+    s_nact = n;
+  }
+  __syncthreads();
+  const int nact = s_nact;
 
   // ---- phase 1: LSE and weights, one thread per row
   {
@@ -141,16 +151,19 @@ __global__ void __launch_bounds__(kMR) merge_kernel(const __grid_constant__ Merg
   for (int i = warp; i < nrows; i += kMR / 32) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     const size_t rowoff = (hrow0 + i) * kRowBytes + sub * 16;
-    for (int p0 = 0; p0 < P; p0 += SPW * kUnroll) {
+    // Only the partitions that contribute a state are visited (a composed cache leaves
+    // most slots of a reused group empty), so every load slot in flight is a real one.
+    for (int k0 = 0; k0 < nact; k0 += SPW * kUnroll) {
       uint4 v[kUnroll];
       float wt[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        const int p = p0 + u * SPW + slot;
+        const int k = k0 + u * SPW + slot;
         wt[u] = 0.0f;
         v[u] = make_uint4(0, 0, 0, 0);
-        const int e = p < P ? s_state[p] : -1;
-        if (e != -1) {
+        if (k < nact) {
+          const int p = s_act[k];
+          const int e = s_state[p];
           wt[u] = sW[p * (kMR + 1) + i];
           const uint8_t* base = e >= 0 ? of : oc;
           v[u] = __ldg(reinterpret_cast<const uint4*>(base + (e >= 0 ? e : -e - 2) * BHN * kRowBytes + rowoff));
@@ -196,16 +209,130 @@ __global__ void __launch_bounds__(kMR) importance_kernel(const __grid_constant__
   }
 }
 
-__global__ void __launch_bounds__(128) reduce_w_kernel(const __grid_constant__ ReduceWParams prm) {
-  const int qg = blockIdx.x;
-  const int b0 = prm.blk_start[qg], b1 = prm.blk_start[qg + 1];
-  for (int p = threadIdx.x; p < prm.P; p += blockDim.x) {
-    double s = 0.0;
-    for (int bh = 0; bh < prm.BH; ++bh)
-      for (int b = b0; b < b1; ++b)
-        s += prm.w_partial[(static_cast<size_t>(bh) * prm.blocks_per_bh + b) * prm.P + p];
-    prm.w[qg * prm.P + p] = static_cast<float>(s * prm.inv_count[qg]);
+// One block per (query group, partition): the threads stride over the group's (b*h,
+// row block) partial sums in a fixed assignment and add them in fp64, then a fixed-shape
+// tree adds the threads' sums -- the same order on every run (deterministic).
+constexpr int kRT = 256;
+
+__global__ void __launch_bounds__(kRT) reduce_w_kernel(const __grid_constant__ ReduceWParams prm) {
+  __shared__ double s_sum[kRT];
+  const int qg = blockIdx.x / prm.P, p = blockIdx.x - qg * prm.P;
+  const int b0 = prm.blk_start[qg], nb = prm.blk_start[qg + 1] - b0;
+  const long long E = static_cast<long long>(prm.BH) * nb;
+  double acc = 0.0;
+  for (long long e = threadIdx.x; e < E; e += kRT) {
+    const long long bh = e / nb;
+    const long long b = e - bh * nb;
+    acc += prm.w_partial[(bh * prm.blocks_per_bh + b0 + b) * prm.P + p];
   }
+  s_sum[threadIdx.x] = acc;
+  __syncthreads();
+  for (int off = kRT / 2; off > 0; off >>= 1) {
+    if (static_cast<int>(threadIdx.x) < off) s_sum[threadIdx.x] += s_sum[threadIdx.x + off];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) prm.w[qg * prm.P + p] = static_cast<float>(s_sum[0] * prm.inv_count[qg]);
+}
+
+// Compose: the states of every `factor` consecutive partitions merged into one (DiTango
+// web summary, Methodology 2, "Dynamic Group Compose": coarser cached states without
+// recomputation).  One block per (output group c, b*h, kCR rows): phase 1 forms each
+// row's LSE over the group's partitions and the weights exp(LSE_p - LSE); phase 2 gives
+// every thread 16-byte chunks of kItems (row, chunk) items and, partition by partition,
+// keeps kItems loads in flight.
+constexpr int kCThreads = 256;
+constexpr int kCR = 128;            // rows per compose block
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kCThreads) compose_kernel(const __grid_constant__ ComposeParams prm) {
+  extern __shared__ float sW[];                    // [factor][kCR + 1]
+  constexpr int kCh = D * static_cast<int>(sizeof(T)) / 16;   // chunks per state row
+  constexpr int kItems = kCR * kCh / kCThreads;
+  const int per_c = prm.BH * prm.nblk;
+  const int c = blockIdx.x / per_c;
+  const int rem = blockIdx.x - c * per_c;
+  const int bh = rem / prm.nblk;
+  const int r0 = (rem - bh * prm.nblk) * kCR;
+  const int nrows = min(kCR, prm.N - r0);
+  const int p0 = c * prm.factor;
+  const int np = min(prm.factor, prm.P - p0);
+  const size_t BHN = static_cast<size_t>(prm.BH) * prm.N;
+  const size_t hrow0 = static_cast<size_t>(bh) * prm.N + r0;
+
+  if (threadIdx.x < kCR) {
+    const int t = threadIdx.x;
+    const bool ok = t < nrows;
+    float m = -INFINITY, l = 0.0f;
+    if (ok) {
+      for (int g = 0; g < np; ++g) {
+        const float L = prm.lse_part[(p0 + g) * BHN + hrow0 + t];
+        if (L > m) {
+          l = l * expf(m - L) + 1.0f;
+          m = L;
+        } else if (L > -INFINITY) {
+          l += expf(L - m);
+        }
+      }
+    }
+    const float lse = m > -INFINITY ? m + logf(l) : -INFINITY;
+    if (ok) prm.lse_group[c * BHN + hrow0 + t] = lse;
+    for (int g = 0; g < np; ++g) {
+      float w = 0.0f;
+      if (ok && lse > -INFINITY) w = expf(prm.lse_part[(p0 + g) * BHN + hrow0 + t] - lse);
+      sW[g * (kCR + 1) + t] = w;
+    }
+  }
+  __syncthreads();
+
+  const uint4* src = static_cast<const uint4*>(prm.o_part);
+  uint4* dst = static_cast<uint4*>(prm.o_group);
+  const int nitems = nrows * kCh;
+  float acc[kItems][8];
+#pragma unroll
+  for (int k = 0; k < kItems; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[k][e] = 0.0f;
+  const bool full = nitems == kCR * kCh;            // every item valid: unguarded loads
+  for (int g = 0; g < np; ++g) {
+    const size_t base = ((p0 + g) * BHN + hrow0) * kCh;
+    uint4 v[kItems];
+    if (full) {
+#pragma unroll
+      for (int k = 0; k < kItems; ++k) v[k] = __ldg(src + base + threadIdx.x + k * kCThreads);
+    } else {
+#pragma unroll
+      for (int k = 0; k < kItems; ++k) {
+        const int idx = threadIdx.x + k * kCThreads;
+        v[k] = idx < nitems ? __ldg(src + base + idx) : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kItems; ++k) {
+      const int idx = threadIdx.x + k * kCThreads;
+      const float w = idx < nitems ? sW[g * (kCR + 1) + idx / kCh] : 0.0f;
+      Acc<T>::add(acc[k], v[k], w);
+    }
+  }
+  const size_t obase = (c * BHN + hrow0) * kCh;
+#pragma unroll
+  for (int k = 0; k < kItems; ++k) {
+    const int idx = threadIdx.x + k * kCThreads;
+    if (idx < nitems) dst[obase + idx] = Acc<T>::pack(acc[k]);
+  }
+}
+
+template <typename T, int D>
+int compose_impl(const ComposeParams& prm, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(prm.factor) * (kCR + 1) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(compose_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  const long long C = (prm.P + prm.factor - 1) / prm.factor;
+  const long long blocks = C * prm.BH * prm.nblk;
+  compose_kernel<T, D><<<static_cast<unsigned>(blocks), kCThreads, smem, st>>>(prm);
+  return static_cast<int>(cudaGetLastError());
 }
 
 template <typename T, int D>
@@ -224,10 +351,16 @@ int merge_impl(const MergeParams& prm, cudaStream_t st) {
 }  // namespace
 
 int merge_rows_per_block() { return kMR; }
+int compose_rows_per_block() { return kCR; }
 
 int launch_merge(const MergeParams& prm, int dtype, cudaStream_t st) {
   if (dtype == PA_BF16) return prm.D == 64 ? merge_impl<__nv_bfloat16, 64>(prm, st) : merge_impl<__nv_bfloat16, 128>(prm, st);
   return prm.D == 64 ? merge_impl<float, 64>(prm, st) : merge_impl<float, 128>(prm, st);
+}
+
+int launch_compose(const ComposeParams& prm, int dtype, int D, cudaStream_t st) {
+  if (dtype == PA_BF16) return D == 64 ? compose_impl<__nv_bfloat16, 64>(prm, st) : compose_impl<__nv_bfloat16, 128>(prm, st);
+  return D == 64 ? compose_impl<float, 64>(prm, st) : compose_impl<float, 128>(prm, st);
 }
 
 int launch_importance(const ImportanceParams& prm, cudaStream_t st) {
@@ -237,7 +370,7 @@ int launch_importance(const ImportanceParams& prm, cudaStream_t st) {
 }
 
 int launch_reduce_w(const ReduceWParams& prm, cudaStream_t st) {
-  reduce_w_kernel<<<prm.QG, 128, 0, st>>>(prm);
+  reduce_w_kernel<<<prm.QG * prm.P, kRT, 0, st>>>(prm);
   return static_cast<int>(cudaGetLastError());
 }
 

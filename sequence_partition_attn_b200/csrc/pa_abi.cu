@@ -390,36 +390,23 @@ int pa_compose_states(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, i
   int rc = check_device(ctx);
   if (rc) return rc;
   const long long BH = static_cast<long long>(B) * H;
-  const size_t BHN = static_cast<size_t>(BH) * N;
-  const size_t row_bytes = static_cast<size_t>(D) * (dtype == PA_BF16 ? 2 : 4);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // One merge over each group's partitions: every row is one query group, all fresh.
-  for (int c = 0; c * factor < P; ++c) {
-    const int np = factor < P - c * factor ? factor : P - c * factor;
-    pa::MergeParams prm;
-    memset(&prm, 0, sizeof prm);
-    prm.o_fresh = static_cast<const uint8_t*>(o_part) + static_cast<size_t>(c) * factor * BHN * row_bytes;
-    prm.lse_fresh = lse_part + static_cast<size_t>(c) * factor * BHN;
-    prm.o = static_cast<uint8_t*>(o_group) + static_cast<size_t>(c) * BHN * row_bytes;
-    prm.lse = lse_group + static_cast<size_t>(c) * BHN;
-    prm.BH = (int)BH;
-    prm.N = N;
-    prm.D = D;
-    prm.P = np;
-    prm.G = np;
-    prm.QG = 1;
-    prm.qg_row0[0] = 0;
-    prm.qg_row0[1] = N;
-    for (int p = 0; p < np; ++p) prm.fresh_bits[0][p >> 5] |= 1u << (p & 31);
-    const int rpb = pa::merge_rows_per_block();
-    prm.blocks_per_bh = (N + rpb - 1) / rpb;
-    prm.blk_start[0] = 0;
-    prm.blk_start[1] = prm.blocks_per_bh;
-    if (BH * prm.blocks_per_bh > 0x7fffffffLL) return fail(ctx, PA_EINVAL, "too many row blocks");
-    int e = pa::launch_merge(prm, dtype, st);
-    if (e) return cuda_fail(ctx, e, "compose launch");
-  }
-  return PA_OK;
+  pa::ComposeParams prm;
+  memset(&prm, 0, sizeof prm);
+  prm.o_part = o_part;
+  prm.lse_part = lse_part;
+  prm.o_group = o_group;
+  prm.lse_group = lse_group;
+  prm.BH = (int)BH;
+  prm.N = N;
+  prm.P = P;
+  prm.factor = factor;
+  const int rpb = pa::compose_rows_per_block();
+  prm.nblk = (N + rpb - 1) / rpb;
+  const long long C = (P + factor - 1) / factor;
+  if (C * BH * prm.nblk > 0x7fffffffLL || BH > 0x7fffffffLL) return fail(ctx, PA_EINVAL, "too many row blocks");
+  int e = pa::launch_compose(prm, dtype, D, st);
+  return e ? cuda_fail(ctx, e, "compose launch") : PA_OK;
 }
 
 int pa_importance(pa_ctx* ctx, int B, int H, int N, int P, int G, const int32_t* part_off,

@@ -303,6 +303,15 @@ __device__ __forceinline__ float fast_log2(float x) {
 }  // namespace pa
 
 namespace pa {
+struct ComposeParams {
+  const void* o_part;             // [P][B][H][N][D]
+  const float* lse_part;          // [P][B][H][N]
+  void* o_group;                  // [C][B][H][N][D], C = ceil(P / factor)
+  float* lse_group;               // [C][B][H][N]
+  int BH, N, P, factor;
+  int nblk;                       // 128-row blocks per (b, h)
+};
+
 struct DriftParams {
   const void* o_new;              // [P][B][H][N][D]
   const void* o_ref;              // [P][B][H][N][D]

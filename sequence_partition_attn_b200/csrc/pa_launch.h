@@ -19,6 +19,9 @@ int merge_rows_per_block();
 int launch_importance(const ImportanceParams& prm, cudaStream_t st);
 int launch_reduce_w(const ReduceWParams& prm, cudaStream_t st);
 
+int compose_rows_per_block();
+int launch_compose(const ComposeParams& prm, int dtype, int D, cudaStream_t st);
+
 int drift_rows_per_block();
 int launch_drift(const DriftParams& prm, int dtype, int D, cudaStream_t st);
 int launch_reduce_pair(const ReducePairParams& prm, cudaStream_t st);
