@@ -135,12 +135,20 @@ def barrier(ws):
 
 
 def max_over_ranks(x, ws):
+    """Max of a host scalar over the ranks (NCCL on the GPUs; gloo groups reduce on the host)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(ws, units_per_step, steps, elapsed_ms_max):
+    """Whole-job throughput of `ws` replicas that each processed `units_per_step` per step
+    for `steps` steps, timed by the slowest rank: units per second over all ranks."""
+    return ws * units_per_step * steps / (elapsed_ms_max / 1e3)
 
 
 # ------------------------------------------------------------------ traffic from the ncu summary
@@ -295,7 +303,7 @@ def run_ours(args, ws, rank, local):
     merge_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     elapsed_ms = max_over_ranks(elapsed_ms, ws)
     ms_per_step = elapsed_ms / K
-    value = ws * step.flops * K / (elapsed_ms / 1e3) / 1e12
+    value = replica_throughput(ws, step.flops, K, elapsed_ms) / 1e12
     pk, pk_kind = peaks()
     attn_tflops = step.flops / (attn_ms / 1e3) / 1e12
     merge_gbs = step.merge_bytes / (merge_ms / 1e3) / 1e9
@@ -330,7 +338,7 @@ def run_ours(args, ws, rank, local):
         torch.cuda.synchronize()
         barrier(ws)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws)
-        e2e = {"value": ws * step.flops * K / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": replica_throughput(ws, step.flops, K, e2e_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K}
         del hq, hk, hv, ho, hl, hw
     # ---- dynamic group compose: the cache composed per KV group, merged without importance

@@ -505,7 +505,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                          make_float2(0.f, 0.f)};
         {
           uint32_t w[32];
-          if (nvalid == kBN) exp_pack_half<true, 0>(s, m, sl2, acc, w);
+          // With every exponential on MUFU (kPolyPairs == 0) masked keys need no
+          // separate path: one copy of the loop keeps the hot code small.
+          if (kPolyPairs == 0 || nvalid == kBN) exp_pack_half<true, 0>(s, m, sl2, acc, w);
           else exp_pack_half<false, 0>(s, m, sl2, acc, w);
           tmem_st32(tS + 0, w);
           tmem_wait_st();
@@ -514,7 +516,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         {
           uint32_t w[32];
-          if (nvalid == kBN) exp_pack_half<true, 1>(s, m, sl2, acc, w);
+          // With every exponential on MUFU (kPolyPairs == 0) masked keys need no
+          // separate path: one copy of the loop keeps the hot code small.
+          if (kPolyPairs == 0 || nvalid == kBN) exp_pack_half<true, 1>(s, m, sl2, acc, w);
           else exp_pack_half<false, 1>(s, m, sl2, acc, w);
           tmem_st32(tS + 32, w);
           tmem_wait_st();
