@@ -74,17 +74,77 @@ class AttentionStep:
         pa_partition_attn(self.ctx, self.q, k_prev, v_prev, self.part_off, self.G, None,
                           self.o_cached, self.lse_cached, stream=stream)
 
-    def attention(self, stream=None):
-        pa_partition_attn(self.ctx, self.q, self.k, self.v, self.part_off, self.G, self.fresh,
+    def attention(self, stream=None, q=None, k=None, v=None):
+        """Fresh states from q, k, v (default: the step's own input buffers)."""
+        pa_partition_attn(self.ctx, self.q if q is None else q, self.k if k is None else k,
+                          self.v if v is None else v, self.part_off, self.G, self.fresh,
                           self.o_fresh, self.lse_fresh, stream=stream)
 
-    def merge(self, stream=None):
+    def merge(self, stream=None, o=None, lse=None, w=None):
+        """Merge into o, lse, w (default: the step's own output buffers)."""
         pa_merge_states(self.ctx, self.part_off, self.G, self.fresh, self.o_fresh, self.lse_fresh,
-                        self.o_cached, self.lse_cached, self.o, self.lse, self.w, stream=stream)
+                        self.o_cached, self.lse_cached, self.o if o is None else o,
+                        self.lse if lse is None else lse, self.w if w is None else w, stream=stream)
 
     def run(self, stream=None):
         self.attention(stream)
         self.merge(stream)
+
+
+class StreamedSteps:
+    """Steps fed from host memory with the copies of neighbouring steps overlapped with
+    compute.  Inputs (Q, K, V) and outputs (O, LSE, w) are double-buffered on the device;
+    host-to-device copies run on one stream, the step on a second, device-to-host copies
+    on a third, so step i's inputs arrive while step i-1 computes and step i-1's outputs
+    leave while step i computes.  Every step still moves its own inputs in and its own
+    outputs out; the intermediate states stay in the step's buffers.
+    """
+
+    def __init__(self, step: AttentionStep):
+        self.step = step
+        two = lambda t: [torch.empty_like(t) for _ in range(2)]          # noqa: E731
+        self.q, self.k, self.v = two(step.q), two(step.k), two(step.v)
+        self.o, self.lse, self.w = two(step.o), two(step.lse), two(step.w)
+        dev = step.q.device
+        self.s_h2d = torch.cuda.Stream(device=dev)
+        self.s_cmp = torch.cuda.Stream(device=dev)
+        self.s_d2h = torch.cuda.Stream(device=dev)
+
+    def run(self, host_inputs, host_outputs, after=None):
+        """host_inputs[i] = (q, k, v) and host_outputs[i] = (o, lse, w): pinned host tensors
+        of step i (an output triple may be reused across steps).  The copies of step 0 wait
+        for stream `after` (default: the current stream).  Returns the event recorded when
+        the last step's outputs have reached the host."""
+        after = torch.cuda.current_stream() if after is None else after
+        start = torch.cuda.Event()
+        start.record(after)
+        n = len(host_inputs)
+        ev_in, ev_cmp, ev_out = [None] * n, [None] * n, [None] * n
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(self.s_h2d):
+                self.s_h2d.wait_event(start)
+                if i >= 2:
+                    self.s_h2d.wait_event(ev_cmp[i - 2])     # step i-2 done with buffer b
+                for d, h in zip((self.q[b], self.k[b], self.v[b]), host_inputs[i]):
+                    d.copy_(h, non_blocking=True)
+                ev_in[i] = torch.cuda.Event()
+                ev_in[i].record(self.s_h2d)
+            with torch.cuda.stream(self.s_cmp):
+                self.s_cmp.wait_event(ev_in[i])
+                if i >= 2:
+                    self.s_cmp.wait_event(ev_out[i - 2])     # outputs of step i-2 have left
+                self.step.attention(self.s_cmp, self.q[b], self.k[b], self.v[b])
+                self.step.merge(self.s_cmp, self.o[b], self.lse[b], self.w[b])
+                ev_cmp[i] = torch.cuda.Event()
+                ev_cmp[i].record(self.s_cmp)
+            with torch.cuda.stream(self.s_d2h):
+                self.s_d2h.wait_event(ev_cmp[i])
+                for h, d in zip(host_outputs[i], (self.o[b], self.lse[b], self.w[b])):
+                    h.copy_(d, non_blocking=True)
+                ev_out[i] = torch.cuda.Event()
+                ev_out[i].record(self.s_d2h)
+        return ev_out[-1]
 
 
 class Trajectory:

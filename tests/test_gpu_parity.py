@@ -380,3 +380,37 @@ def test_state_drift_empty_sequence_and_errors(pa, ctx):
     o = torch.zeros(P, 1, 1, 64, 64, dtype=torch.bfloat16, device=DEV)
     with pytest.raises(pa.PAError, match="PA_EINVAL"):
         pa.pa_state_drift(ctx, W.part_offsets(63, P), G, None, o, o, d2, r2)
+
+
+# --------------------------------------------------------------------------- streamed steps
+def test_streamed_steps_match_serial_steps(pa, ctx):
+    # three steps fed from host memory with overlapped copies give exactly the outputs of
+    # the same steps run one after another
+    from sequence_partition_attn_b200.step import AttentionStep, StreamedSteps
+    wl = W.small_variant(W.workload(2), grid=(3, 45, 80), H=2)
+    t = W.make_qkv(wl)
+    kc, vc = W.make_cached_kv(wl, t["k"], t["v"])
+    off = W.part_offsets(wl.N, wl.P)
+    step = AttentionStep(ctx, wl.B, wl.H, wl.N, wl.D, off, wl.G, W.reuse_mask(wl), device=DEV)
+    step.q.copy_(t["q"].to(DEV))
+    step.fill_cache(kc.to(DEV), vc.to(DEV))
+    inputs = []
+    k, v = t["k"], t["v"]
+    for s in range(3):
+        if s:
+            k, v = W.drift_kv(wl, k, v, s)
+        inputs.append(tuple(x.pin_memory() for x in (t["q"], k, v)))
+    outs = [(torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory(),
+             torch.empty(step.lse.shape).pin_memory(), torch.empty(step.w.shape).pin_memory())
+            for _ in range(3)]
+    streamed = StreamedSteps(step)
+    done = streamed.run(inputs, outs)
+    done.synchronize()
+    ctx.sync_status()
+    for s in range(3):
+        for d, h in zip((step.q, step.k, step.v), inputs[s]):
+            d.copy_(h.to(DEV))
+        step.run()
+        ctx.sync_status()
+        assert torch.equal(outs[s][0].view(torch.int16), step.o.cpu().view(torch.int16)), s
+        assert torch.equal(outs[s][1], step.lse.cpu()) and torch.equal(outs[s][2], step.w.cpu()), s
