@@ -272,6 +272,20 @@ def test_compose_states(pa, ctx, dt, D, N, P, factor):
     assert maxerr(lg.cpu().numpy(), rl) <= 1e-5 + 1e-6 * np.abs(rl[np.isfinite(rl)]).max()
 
 
+def test_compose_with_factor_one_is_the_identity(pa, ctx):
+    # one partition per group: LSE = LSE_p + ln 1 and weight exp(0) = 1, so the composed
+    # states are the partition states bit for bit (empty partition included)
+    N, P = 333, 7
+    off = W.part_offsets(N, P)
+    o, l = _gen_states(9, P, 2, 2, N, 128, torch.bfloat16, empty=[3])
+    og = torch.empty_like(o, device=DEV)
+    lg = torch.empty_like(l, device=DEV)
+    pa.pa_compose_states(ctx, o.to(DEV), l.to(DEV), 1, og, lg)
+    ctx.sync_status()
+    assert torch.equal(og.cpu().view(torch.int16), o.view(torch.int16))
+    assert torch.equal(lg.cpu(), l)
+
+
 def test_merge_with_composed_cache_against_oracle(pa, ctx):
     # seeded states (generated on the host) for both sides
     N, P, G, D, H = 2900, 32, 4, 128, 2
