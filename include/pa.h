@@ -57,7 +57,11 @@
  * retains caller memory past the call.  A pa_ctx owns only its own device workspace and
  * an error-status word.  Calls are asynchronous on the given stream (a cudaStream_t
  * passed as void*; NULL = the legacy default stream): they validate, enqueue kernels
- * and return.  No call synchronises except pa_sync_status.
+ * and return.  No call synchronises except pa_sync_status, and a call that first needs a
+ * larger workspace (cudaFree of the old one and cudaMalloc synchronise the device).  The
+ * calls that use the workspace -- pa_merge_states with w, pa_importance, pa_state_drift
+ * -- share it, so on one context they must not overlap on the GPU (issue them on one
+ * stream, or use a context per stream).
  *
  * Errors.  Every call returns PA_OK (0) or a negative status; pa_last_error gives a
  * one-line message for the last failure on that context (thread-unsafe per context).
@@ -159,8 +163,10 @@ typedef struct {
  * fresh[qg][p/G] != 0, else from the cached arrays; write LSE(i), O(i) (fp32 math, O
  * rounded to dtype) and, if w != NULL, overwrite w with the importance of the merged
  * states.  With cached_per_group, a reused KV group contributes its one composed cached
- * state instead of G per-partition states (fewer bytes read per row).  Uses a context workspace of about 4*P*ceil(B*H*N/256) bytes, allocated on
- * first need.  Errors: PA_EINVAL, PA_EALIGN, PA_EUNSUPPORTED, PA_ENOMEM, PA_ECUDA. */
+ * state instead of G per-partition states (fewer bytes read per row).  With w != NULL it
+ * uses a context workspace of 4*P bytes per 128-row block of each query group of each
+ * (b, h) -- about 4*P*B*H*N/128 bytes -- allocated on first need and grown, never shrunk.
+ * Errors: PA_EINVAL, PA_EALIGN, PA_EUNSUPPORTED, PA_ENOMEM, PA_ECUDA. */
 int pa_merge_states(pa_ctx* ctx, const pa_merge_desc* desc, void* stream);
 
 /* ---------------------------------------------------------------- group compose */
