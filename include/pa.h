@@ -232,6 +232,17 @@ int pa_state_drift(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int 
                    const int32_t* part_off, const uint8_t* sel, const void* o_new,
                    const void* o_ref, float* d2, float* r2, void* stream);
 
+/* ---------------------------------------------------------------- bounded-wait self-test */
+/* Library diagnostics; the pages have no counterpart.  Every pipeline barrier wait in the
+ * kernels gives up after a time limit instead of spinning for ever, records PA_ETIMEOUT in
+ * the context status word and stops the block.  This call launches a one-block kernel
+ * whose two waits (the whole-warp form and the per-thread form) wait on a barrier nothing
+ * completes, with a limit of `seconds` (0 < seconds <= 2): both give up within the limit,
+ * and a following pa_sync_status returns PA_ETIMEOUT (and clears it), after which the
+ * context is usable again.  No fault and no hang are involved.
+ * Errors: PA_EINVAL, PA_ECUDA. */
+int pa_selftest_wait(pa_ctx* ctx, double seconds, void* stream);
+
 /* ---------------------------------------------------------------- relayout */
 /* dst[h][n][:] = src[n][h][:] for the tokens of sequence chunk `chunk` of `n_chunks`
  * (chunk c covers n in [c*ceil(N/n_chunks), min((c+1)*ceil(N/n_chunks), N)));

@@ -23,7 +23,8 @@ import numpy as np
 __all__ = [
     "PA_F32", "PA_BF16", "PAError", "Context", "lib", "lib_path",
     "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head",
-    "pa_merge_states_noalloc", "pa_compose_states", "pa_state_drift", "EXPORTED", "select_fresh",
+    "pa_merge_states_noalloc", "pa_compose_states", "pa_state_drift", "pa_selftest_wait", "EXPORTED",
+    "select_fresh",
     "predict_fresh",
 ]
 
@@ -33,7 +34,7 @@ _ERRORS = {-1: "PA_EINVAL", -2: "PA_EALIGN", -3: "PA_EUNSUPPORTED", -4: "PA_ENOM
            -5: "PA_ECUDA", -6: "PA_ETIMEOUT"}
 EXPORTED = ("pa_init", "pa_destroy", "pa_last_error", "pa_sync_status", "pa_version",
             "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head",
-            "pa_merge_states_noalloc", "pa_compose_states", "pa_state_drift")
+            "pa_merge_states_noalloc", "pa_compose_states", "pa_state_drift", "pa_selftest_wait")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -94,8 +95,9 @@ def lib():
         L.pa_compose_states.argtypes = [vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
         L.pa_relayout_seq2head.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, vp]
         L.pa_state_drift.argtypes = [vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp]
+        L.pa_selftest_wait.argtypes = [vp, ctypes.c_double, vp]
         for f in ("pa_init", "pa_sync_status", "pa_partition_attn", "pa_merge_states", "pa_merge_states_noalloc",
-                  "pa_compose_states", "pa_state_drift",
+                  "pa_compose_states", "pa_state_drift", "pa_selftest_wait",
                   "pa_importance", "pa_relayout_seq2head"):
             getattr(L, f).restype = ci
         _LIB = L
@@ -246,6 +248,12 @@ def pa_state_drift(ctx: Context, part_off, G, sel, o_new, o_ref, d2, r2, stream=
                                          off.ctypes.data, None if sl is None else sl.ctypes.data,
                                          o_new.data_ptr(), o_ref.data_ptr(), d2.data_ptr(),
                                          r2.data_ptr(), _stream(stream)))
+
+
+def pa_selftest_wait(ctx: Context, seconds=0.05, stream=None):
+    """Launch the bounded-wait self-test: a wait that nothing completes gives up after
+    `seconds`; the next ctx.sync_status() raises PAError with code PA_ETIMEOUT."""
+    _check(ctx.ptr, lib().pa_selftest_wait(ctx.ptr, float(seconds), _stream(stream)))
 
 
 def pa_relayout_seq2head(ctx: Context, src, dst, n_chunks=1, chunk=-1, stream=None):

@@ -506,6 +506,16 @@ int pa_state_drift(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int 
   return e ? cuda_fail(ctx, e, "drift reduce launch") : PA_OK;
 }
 
+int pa_selftest_wait(pa_ctx* ctx, double seconds, void* stream) {
+  if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
+  if (!(seconds > 0.0 && seconds <= 2.0)) return fail(ctx, PA_EINVAL, "seconds=%g outside (0, 2]", seconds);
+  int rc = check_device(ctx);
+  if (rc) return rc;
+  int e = pa::launch_wait_selftest(ctx->d_status, static_cast<uint64_t>(seconds * 1e9),
+                                   static_cast<cudaStream_t>(stream));
+  return e ? cuda_fail(ctx, e, "wait selftest launch") : PA_OK;
+}
+
 int pa_relayout_seq2head(pa_ctx* ctx, const void* src, void* dst, int N, int H, int D, int elem_bytes,
                          int n_chunks, int chunk, void* stream) {
   if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");

@@ -22,6 +22,8 @@ int launch_reduce_w(const ReduceWParams& prm, cudaStream_t st);
 int compose_rows_per_block();
 int launch_compose(const ComposeParams& prm, int dtype, int D, cudaStream_t st);
 
+int launch_wait_selftest(int* status, uint64_t limit_ns, cudaStream_t st);
+
 int drift_rows_per_block();
 int launch_drift(const DriftParams& prm, int dtype, int D, cudaStream_t st);
 int launch_reduce_pair(const ReducePairParams& prm, cudaStream_t st);

@@ -64,6 +64,9 @@ def test_null_context_is_rejected(lib):
     assert lib.pa_merge_states(None, None, None) == -1
     assert lib.pa_importance(None, 1, 1, 1, 1, 1, None, None, None, None, None) == -1
     assert lib.pa_relayout_seq2head(None, None, None, 1, 1, 8, 2, 1, -1, None) == -1
+    assert lib.pa_compose_states(None, 1, 1, 1, 1, 64, 1, 1, None, None, None, None, None) == -1
+    assert lib.pa_state_drift(None, 1, 1, 1, 1, 64, 1, 1, None, None, None, None, None, None, None) == -1
+    assert lib.pa_selftest_wait(None, 0.01, None) == -1
     assert lib.pa_sync_status(None, None) == -1
     assert b"ctx" in lib.pa_last_error(None)
     lib.pa_destroy(None)                   # no-op

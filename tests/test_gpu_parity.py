@@ -428,3 +428,20 @@ def test_streamed_steps_match_serial_steps(pa, ctx):
         ctx.sync_status()
         assert torch.equal(outs[s][0].view(torch.int16), step.o.cpu().view(torch.int16)), s
         assert torch.equal(outs[s][1], step.lse.cpu()) and torch.equal(outs[s][2], step.w.cpu()), s
+
+
+# --------------------------------------------------------------------------- bounded waits
+def test_bounded_wait_gives_up_reports_and_recovers(pa, ctx):
+    # a wait on a barrier nothing completes gives up after 50 ms, the status word says
+    # PA_ETIMEOUT once, and the context keeps working afterwards
+    import time
+    t0 = time.time()
+    pa.pa_selftest_wait(ctx, 0.05)
+    with pytest.raises(pa.PAError, match="PA_ETIMEOUT"):
+        ctx.sync_status()
+    assert time.time() - t0 < 10.0
+    ctx.sync_status()                     # read and cleared
+    with pytest.raises(pa.PAError, match="PA_EINVAL"):
+        pa.pa_selftest_wait(ctx, 3.0)     # limits above 2 s are refused
+    wl = W.small_variant(W.workload(1), grid=(1, 20, 23), H=1, P=4, mask="all")
+    _check_case(pa, ctx, wl)
