@@ -247,7 +247,7 @@ int pa_selftest_wait(pa_ctx* ctx, double seconds, void* stream);
 /* dst[h][n][:] = src[n][h][:] for the tokens of sequence chunk `chunk` of `n_chunks`
  * (chunk c covers n in [c*ceil(N/n_chunks), min((c+1)*ceil(N/n_chunks), N)));
  * chunk = -1 moves every chunk.  A bit-exact copy: D*elem_bytes must be a multiple of
- * 16.  Errors: PA_EINVAL, PA_EALIGN, PA_ECUDA. */
+ * 16 and at most 16384.  Errors: PA_EINVAL, PA_EALIGN, PA_EUNSUPPORTED, PA_ECUDA. */
 int pa_relayout_seq2head(pa_ctx* ctx, const void* src, void* dst, int N, int H, int D,
                          int elem_bytes, int n_chunks, int chunk, void* stream);
 

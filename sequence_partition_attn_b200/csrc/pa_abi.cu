@@ -524,6 +524,7 @@ int pa_relayout_seq2head(pa_ctx* ctx, const void* src, void* dst, int N, int H, 
     return fail(ctx, PA_EINVAL, "elem_bytes=%d", elem_bytes);
   const long long row_bytes = static_cast<long long>(D) * elem_bytes;
   if (row_bytes % 16 != 0) return fail(ctx, PA_EINVAL, "D*elem_bytes=%lld is not a multiple of 16", row_bytes);
+  if (row_bytes > 16384) return fail(ctx, PA_EUNSUPPORTED, "D*elem_bytes=%lld above 16384", row_bytes);
   if (n_chunks < 1) return fail(ctx, PA_EINVAL, "n_chunks=%d", n_chunks);
   if (chunk < -1 || chunk >= n_chunks) return fail(ctx, PA_EINVAL, "chunk=%d outside [-1, %d)", chunk, n_chunks);
   if (N == 0) return PA_OK;

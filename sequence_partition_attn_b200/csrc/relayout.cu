@@ -15,28 +15,44 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;
 
-__global__ void __launch_bounds__(kThreads) relayout_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
-                                                            long long n0, long long total, int N, int H,
-                                                            int ppr) {
-  const long long stride = static_cast<long long>(gridDim.x) * kThreads;
-  const long long src0 = n0 * H * ppr;
-  for (long long base = static_cast<long long>(blockIdx.x) * kThreads + threadIdx.x; base < total;
-       base += stride * kUnroll) {
+// Thread t of the grid copies piece (t mod ppr) of rows r, r + dr, r + 2 dr, ... where
+// r = t / ppr and dr = grid threads / ppr (the block size is a multiple of ppr, so every
+// thread keeps its piece).  Row r = n' * H + h is token n0 + n', head h; (n', h) of each of the
+// kUnroll rows in flight advance by a constant step with one carry, so the loop does no
+// division.
+__global__ void __launch_bounds__(1024) relayout_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                        long long n0, long long rows, int N, int H, int ppr) {
+  const long long gthreads = static_cast<long long>(gridDim.x) * blockDim.x;
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int piece = static_cast<int>(t % ppr);
+  const long long dr = gthreads / ppr;                 // rows per grid step
+  const long long step = dr * kUnroll;                 // rows per loop iteration
+  const long long step_n = step / H;
+  const int step_h = static_cast<int>(step % H);
+  long long r[kUnroll], n[kUnroll];
+  int h[kUnroll];
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) {
+    r[u] = t / ppr + u * dr;
+    n[u] = r[u] / H;
+    h[u] = static_cast<int>(r[u] - n[u] * H);
+  }
+  const uint4* s0 = src + n0 * H * ppr + piece;
+  uint4* d0 = dst + n0 * ppr + piece;
+  while (r[0] < rows) {
     uint4 v[kUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const long long idx = base + u * stride;
-      if (idx < total) v[u] = __ldg(src + src0 + idx);
-    }
+    for (int u = 0; u < kUnroll; ++u)
+      if (r[u] < rows) v[u] = __ldg(s0 + r[u] * ppr);
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const long long idx = base + u * stride;
-      if (idx < total) {
-        const long long rowi = idx / ppr;
-        const int piece = static_cast<int>(idx - rowi * ppr);
-        const long long n = n0 + rowi / H;
-        const int h = static_cast<int>(rowi % H);
-        dst[(static_cast<long long>(h) * N + n) * ppr + piece] = v[u];
+      if (r[u] < rows) d0[(static_cast<long long>(h[u]) * N + n[u]) * ppr] = v[u];
+      r[u] += step;
+      n[u] += step_n;
+      h[u] += step_h;
+      if (h[u] >= H) {
+        h[u] -= H;
+        ++n[u];
       }
     }
   }
@@ -46,14 +62,16 @@ __global__ void __launch_bounds__(kThreads) relayout_kernel(const uint4* __restr
 
 int launch_relayout(const void* src, void* dst, long long n0, long long n1, int N, int H, int row_bytes,
                     int sm_count, cudaStream_t st) {
-  const int ppr = row_bytes / 16;
-  const long long total = (n1 - n0) * H * ppr;
-  if (total <= 0) return 0;
-  long long blocks = (total + kThreads * kUnroll - 1) / (kThreads * kUnroll);
+  const int ppr = row_bytes / 16;                    // 16-byte pieces per row
+  if (ppr < 1 || ppr > 1024) return static_cast<int>(cudaErrorInvalidValue);
+  const int threads = ppr >= kThreads ? ppr : (kThreads / ppr) * ppr;   // a multiple of ppr
+  const long long rows = (n1 - n0) * H;
+  if (rows <= 0) return 0;
+  long long blocks = (rows * ppr + static_cast<long long>(threads) * kUnroll - 1) / (static_cast<long long>(threads) * kUnroll);
   const long long cap = static_cast<long long>(sm_count) * 8;
   if (blocks > cap) blocks = cap;
-  relayout_kernel<<<static_cast<unsigned>(blocks), kThreads, 0, st>>>(
-      static_cast<const uint4*>(src), static_cast<uint4*>(dst), n0, total, N, H, ppr);
+  relayout_kernel<<<static_cast<unsigned>(blocks), threads, 0, st>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), n0, rows, N, H, ppr);
   return static_cast<int>(cudaGetLastError());
 }
 

@@ -33,7 +33,11 @@ DEV = "cuda:0"
 @pytest.mark.parametrize("N,H,D,dt,chunks", [(1000, 3, 128, torch.bfloat16, 16),
                                                (777, 5, 64, torch.float32, 3),
                                                (64, 1, 8, torch.bfloat16, 1),
-                                               (7200 * 2, 24, 128, torch.bfloat16, 16)])
+                                               (7200 * 2, 24, 128, torch.bfloat16, 16),
+                                               (333, 7, 96, torch.bfloat16, 5),     # 12 pieces per row
+                                               (129, 3, 24, torch.bfloat16, 2),     # 3 pieces per row
+                                               (50, 2, 40, torch.float32, 3),       # 10 pieces per row
+                                               (40, 3, 2048, torch.float32, 4)])    # 512 pieces per row
 def test_relayout_bit_exact(pa, ctx, N, H, D, dt, chunks):
     g = torch.Generator().manual_seed(N + H)
     src = torch.randn(N, H, D, generator=g).to(dt)
@@ -49,6 +53,12 @@ def test_relayout_bit_exact(pa, ctx, N, H, D, dt, chunks):
     pa.pa_relayout_seq2head(ctx, s, dst2, n_chunks=chunks, chunk=-1)   # all at once
     ctx.sync_status()
     assert np.array_equal(dst2.cpu().view(bits).numpy(), ref)
+
+
+def test_relayout_rejects_rows_above_16_kib(pa, ctx):
+    src = torch.zeros(4, 1, 8192, dtype=torch.float32, device=DEV)
+    with pytest.raises(pa.PAError, match="PA_EUNSUPPORTED"):
+        pa.pa_relayout_seq2head(ctx, src, src.view(1, 4, 8192))
 
 
 def test_relayout_single_chunk_touches_only_its_rows(pa, ctx):
