@@ -350,16 +350,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (!wait_p(bar(L::P_LO + 0), j & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv<D, 0>(tmem + 256, tmem, dv, kIdPV, first);
+          // K(j+1) is checked while P hi is still being produced, so that PV hi and the
+          // next S issue back to back once it arrives.
+          if (more && !mbar_wait_warp(bar(L::K_FULL + s1), ((j + 1) / kStages) & 1, abort_flag, status)) {
+            ok = false;
+            break;
+          }
           if (!wait_p(bar(L::P_HI + 0), j & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv<D, 1>(tmem + 256, tmem, dv, kIdPV, first);
           commit(L::O_DONE + 0);
           if (more) {
-            if (!mbar_wait_warp(bar(L::K_FULL + s1), ((j + 1) / kStages) & 1, abort_flag, status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
             issue_s<D>(tmem, dq0, dk, kIdS);
             commit(L::S_FULL + 0);
           }
