@@ -63,6 +63,11 @@
  * -- share it, so on one context they must not overlap on the GPU (issue them on one
  * stream, or use a context per stream).
  *
+ * Debug.  With PA_DEBUG set (not "0") in the environment when pa_init runs, every call on
+ * that context synchronises its stream after launching and returns what pa_sync_status
+ * would (PA_ECUDA for a launch or runtime error, PA_ETIMEOUT for a device-side wait that
+ * gave up).
+ *
  * Errors.  Every call returns PA_OK (0) or a negative status; pa_last_error gives a
  * one-line message for the last failure on that context (thread-unsafe per context).
  * Validation happens before anything is enqueued: on error nothing was launched.

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -17,6 +18,7 @@ struct pa_ctx {
   int device = -1;
   int sm_count = 0;
   int* d_status = nullptr;         // device status word (bounded-wait give-ups)
+  bool debug = false;              // PA_DEBUG: synchronise and check after every call
   void* ws = nullptr;              // workspace for per-block importance sums
   size_t ws_bytes = 0;
   std::string err;
@@ -214,6 +216,8 @@ int pa_init(int device, pa_ctx** out) {
   pa_ctx* ctx = new pa_ctx();
   ctx->device = device;
   ctx->sm_count = prop.multiProcessorCount;
+  const char* dbg = getenv("PA_DEBUG");
+  ctx->debug = dbg && *dbg && strcmp(dbg, "0") != 0;
   if (cudaMalloc(&ctx->d_status, sizeof(int)) != cudaSuccess || cudaMemset(ctx->d_status, 0, sizeof(int)) != cudaSuccess) {
     cudaGetLastError();
     if (ctx->d_status) cudaFree(ctx->d_status);
@@ -247,7 +251,7 @@ int pa_sync_status(pa_ctx* ctx, void* stream) {
   return PA_OK;
 }
 
-int pa_partition_attn(pa_ctx* ctx, const pa_attn_desc* d, void* stream) {
+static int pa_partition_attn_impl(pa_ctx* ctx, const pa_attn_desc* d, void* stream) {
   if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
   if (!d) return fail(ctx, PA_EINVAL, "desc is NULL");
   if (d->dtype != PA_BF16 && d->dtype != PA_F32) return fail(ctx, PA_EUNSUPPORTED, "dtype %d", (int)d->dtype);
@@ -311,7 +315,7 @@ int pa_partition_attn(pa_ctx* ctx, const pa_attn_desc* d, void* stream) {
   return e ? cuda_fail(ctx, e, "attn_f32 launch") : PA_OK;
 }
 
-int pa_merge_states(pa_ctx* ctx, const pa_merge_desc* d, void* stream) {
+static int pa_merge_states_impl(pa_ctx* ctx, const pa_merge_desc* d, void* stream) {
   if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
   if (!d) return fail(ctx, PA_EINVAL, "desc is NULL");
   if (d->dtype != PA_BF16 && d->dtype != PA_F32) return fail(ctx, PA_EUNSUPPORTED, "dtype %d", (int)d->dtype);
@@ -374,7 +378,7 @@ int pa_merge_states(pa_ctx* ctx, const pa_merge_desc* d, void* stream) {
   return PA_OK;
 }
 
-int pa_compose_states(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int P, int factor,
+static int pa_compose_states_impl(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int P, int factor,
                       const void* o_part, const float* lse_part, void* o_group, float* lse_group,
                       void* stream) {
   if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
@@ -409,7 +413,7 @@ int pa_compose_states(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, i
   return e ? cuda_fail(ctx, e, "compose launch") : PA_OK;
 }
 
-int pa_importance(pa_ctx* ctx, int B, int H, int N, int P, int G, const int32_t* part_off,
+static int pa_importance_impl(pa_ctx* ctx, int B, int H, int N, int P, int G, const int32_t* part_off,
                   const float* lse_part, const float* lse, float* w, void* stream) {
   if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
   if (B < 1 || H < 1 || N < 0) return fail(ctx, PA_EINVAL, "B=%d H=%d N=%d", B, H, N);
@@ -445,7 +449,7 @@ int pa_importance(pa_ctx* ctx, int B, int H, int N, int P, int G, const int32_t*
   return launch_reduce(ctx, t, prm.blk_start, bpb, (int)BH, w, st);
 }
 
-int pa_state_drift(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int P, int G,
+static int pa_state_drift_impl(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int P, int G,
                    const int32_t* part_off, const uint8_t* sel, const void* o_new, const void* o_ref,
                    float* d2, float* r2, void* stream) {
   if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
@@ -506,7 +510,7 @@ int pa_state_drift(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int 
   return e ? cuda_fail(ctx, e, "drift reduce launch") : PA_OK;
 }
 
-int pa_selftest_wait(pa_ctx* ctx, double seconds, void* stream) {
+static int pa_selftest_wait_impl(pa_ctx* ctx, double seconds, void* stream) {
   if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
   if (!(seconds > 0.0 && seconds <= 2.0)) return fail(ctx, PA_EINVAL, "seconds=%g outside (0, 2]", seconds);
   int rc = check_device(ctx);
@@ -516,7 +520,7 @@ int pa_selftest_wait(pa_ctx* ctx, double seconds, void* stream) {
   return e ? cuda_fail(ctx, e, "wait selftest launch") : PA_OK;
 }
 
-int pa_relayout_seq2head(pa_ctx* ctx, const void* src, void* dst, int N, int H, int D, int elem_bytes,
+static int pa_relayout_seq2head_impl(pa_ctx* ctx, const void* src, void* dst, int N, int H, int D, int elem_bytes,
                          int n_chunks, int chunk, void* stream) {
   if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
   if (N < 0 || H < 1 || D < 1) return fail(ctx, PA_EINVAL, "N=%d H=%d D=%d", N, H, D);
@@ -541,6 +545,48 @@ int pa_relayout_seq2head(pa_ctx* ctx, const void* src, void* dst, int N, int H, 
   int e = pa::launch_relayout(src, dst, n0, n1, N, H, static_cast<int>(row_bytes), ctx->sm_count,
                               static_cast<cudaStream_t>(stream));
   return e ? cuda_fail(ctx, e, "relayout launch") : PA_OK;
+}
+
+// With PA_DEBUG set when the context was created, every call synchronises its stream after
+// launching and returns what pa_sync_status finds (a launch or runtime error, or a
+// bounded device-side wait that gave up).
+static int debug_finish(pa_ctx* ctx, void* stream, int rc) {
+  if (rc != PA_OK || !ctx || !ctx->debug) return rc;
+  return pa_sync_status(ctx, stream);
+}
+
+int pa_partition_attn(pa_ctx* ctx, const pa_attn_desc* d, void* stream) {
+  return debug_finish(ctx, stream, pa_partition_attn_impl(ctx, d, stream));
+}
+
+int pa_merge_states(pa_ctx* ctx, const pa_merge_desc* d, void* stream) {
+  return debug_finish(ctx, stream, pa_merge_states_impl(ctx, d, stream));
+}
+
+int pa_compose_states(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int P, int factor,
+                      const void* o_part, const float* lse_part, void* o_group, float* lse_group,
+                      void* stream) {
+  return debug_finish(ctx, stream, pa_compose_states_impl(ctx, dtype, B, H, N, D, P, factor, o_part, lse_part, o_group, lse_group, stream));
+}
+
+int pa_importance(pa_ctx* ctx, int B, int H, int N, int P, int G, const int32_t* part_off,
+                  const float* lse_part, const float* lse, float* w, void* stream) {
+  return debug_finish(ctx, stream, pa_importance_impl(ctx, B, H, N, P, G, part_off, lse_part, lse, w, stream));
+}
+
+int pa_state_drift(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int P, int G,
+                   const int32_t* part_off, const uint8_t* sel, const void* o_new, const void* o_ref,
+                   float* d2, float* r2, void* stream) {
+  return debug_finish(ctx, stream, pa_state_drift_impl(ctx, dtype, B, H, N, D, P, G, part_off, sel, o_new, o_ref, d2, r2, stream));
+}
+
+int pa_relayout_seq2head(pa_ctx* ctx, const void* src, void* dst, int N, int H, int D, int elem_bytes,
+                         int n_chunks, int chunk, void* stream) {
+  return debug_finish(ctx, stream, pa_relayout_seq2head_impl(ctx, src, dst, N, H, D, elem_bytes, n_chunks, chunk, stream));
+}
+
+int pa_selftest_wait(pa_ctx* ctx, double seconds, void* stream) {
+  return debug_finish(ctx, stream, pa_selftest_wait_impl(ctx, seconds, stream));
 }
 
 }  // extern "C"

@@ -455,3 +455,18 @@ def test_bounded_wait_gives_up_reports_and_recovers(pa, ctx):
         pa.pa_selftest_wait(ctx, 3.0)     # limits above 2 s are refused
     wl = W.small_variant(W.workload(1), grid=(1, 20, 23), H=1, P=4, mask="all")
     _check_case(pa, ctx, wl)
+
+
+def test_debug_mode_reports_at_the_call(pa, monkeypatch):
+    # PA_DEBUG at context creation: every call synchronises and returns the status itself
+    monkeypatch.setenv("PA_DEBUG", "1")
+    c = pa.Context(0)
+    try:
+        with pytest.raises(pa.PAError, match="PA_ETIMEOUT"):
+            pa.pa_selftest_wait(c, 0.02)
+        src = torch.randn(64, 2, 64, device=DEV).to(torch.bfloat16)
+        dst = torch.empty(2, 64, 64, dtype=torch.bfloat16, device=DEV)
+        pa.pa_relayout_seq2head(c, src, dst)             # an ordinary call passes through
+        assert torch.equal(dst.cpu(), src.cpu().transpose(0, 1))
+    finally:
+        c.close()
