@@ -214,9 +214,18 @@ def oracle_sample(wl, heads, rows_per_group, seed=5, host=None):
 def cpu_baseline_entry(wl, full_flops, host=None):
     dt, flops, threads, desc = oracle_sample(wl, heads=wl.H, rows_per_group=128, host=host)
     tflops = flops / dt / 1e12
-    return {"value": tflops, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": desc, "seconds": dt,
-            "extrapolated_full_step_s": full_flops / (flops / dt)}
+    entry = {"value": tflops, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+             "sample": desc, "seconds": dt,
+             "extrapolated_full_step_s": full_flops / (flops / dt)}
+    try:                                   # the same oracle on one core, smaller sample
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            dt1, flops1, _, desc1 = oracle_sample(wl, heads=4, rows_per_group=32, seed=6)
+        entry["one_core"] = {"value": flops1 / dt1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                             "sample": desc1, "seconds": dt1}
+    except ImportError:
+        pass
+    return entry
 
 
 # ------------------------------------------------------------------ reference arm
