@@ -181,6 +181,15 @@ def test_bf16_small_cases(pa, ctx, kw):
     _check_case(pa, ctx, wl)
 
 
+def test_bf16_maximum_partition_count(pa, ctx):
+    # P = 128 (the largest table the ABI takes), G = 16, 8 groups of 16 partitions of ~16
+    # keys: every partition is shorter than a key tile; a random group mask
+    wl = W.small_variant(W.workload(1), grid=(1, 40, 50), H=1, P=128, G=16)
+    fresh = (np.random.default_rng(17).random((wl.QG, wl.KG)) < 0.5).astype(np.uint8)
+    np.fill_diagonal(fresh, 1)
+    _check_case(pa, ctx, wl, fresh)
+
+
 def test_fp32_small_ragged_case(pa, ctx):
     wl = W.small_variant(W.workload(0), grid=(1, 13, 23), H=2, P=3, G=1, cache_sigma=0.05,
                          mask="neighbours", D=128)
