@@ -85,15 +85,21 @@ constexpr float kC1 = 0.6932609677314758f;
 constexpr float kC2 = 0.24261093139648438f;
 constexpr float kC3 = 0.05517149344086647f;
 
-// 2^t on the FMA pipe.  t is clamped at -126 so that adding n to the exponent field of
-// 2^f (which lies in [0.70, 1.42]) can never underflow the field.
-__device__ __forceinline__ float poly_exp2(float t) {
-  t = fmaxf(t, -126.0f);
-  const float rnd = t + 12582912.0f;          // 1.5 * 2^23: n = round(t) lands in the low bits
-  const float n = rnd - 12582912.0f;
-  const float f = t - n;
-  const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(rnd) << 23));
+// 2^t for a pair of values on the FMA pipe, with packed fp32x2 arithmetic (one instruction
+// per pair for the rounding, the reduction and the polynomial).  t is clamped at -126 so
+// that adding n to the exponent field of 2^f (which lies in [0.70, 1.42]) can never
+// underflow the field; n = round(t) lands in the low mantissa bits of t + 1.5 * 2^23.
+__device__ __forceinline__ float2 poly_exp2x2(float2 t) {
+  t.x = fmaxf(t.x, -126.0f);
+  t.y = fmaxf(t.y, -126.0f);
+  const float2 rnd = __fadd2_rn(t, make_float2(12582912.0f, 12582912.0f));
+  const float2 n = __fadd2_rn(rnd, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __fadd2_rn(t, make_float2(-n.x, -n.y));
+  float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+  p = __ffma2_rn(p, f, make_float2(kC0, kC0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(rnd.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(rnd.y) << 23)));
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -126,20 +132,6 @@ __device__ __forceinline__ int tile_row0(int key, int k0, int k1) {
   return (key + kBN > k1 && k1 - kBN >= k0) ? k1 - kBN : key;
 }
 
-// The same on a pair of values with packed fp32x2 arithmetic (one instruction per pair
-// for the rounding, the reduction and the polynomial).
-__device__ __forceinline__ float2 poly_exp2x2(float2 t) {
-  t.x = fmaxf(t.x, -126.0f);
-  t.y = fmaxf(t.y, -126.0f);
-  const float2 rnd = __fadd2_rn(t, make_float2(12582912.0f, 12582912.0f));
-  const float2 n = __fadd2_rn(rnd, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = __fadd2_rn(t, make_float2(-n.x, -n.y));
-  float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
-  p = __ffma2_rn(p, f, make_float2(kC0, kC0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(rnd.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(rnd.y) << 23)));
-}
 
 // Next partition >= from that is fresh for query group qg and holds at least one key.
 __device__ __forceinline__ int next_part(const AttnTables& t, int qg, int from) {
