@@ -19,7 +19,7 @@ for Distributed Inference of Diffusion Transformers on GPUs"):
 * a sequence-major layout that a chunked all-to-all turns head-major -- SwiftFusion,
   Methodology 2 (Torus Attention).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * tokens are ordered t-major: n = (t*Hh + h)*W + w;
 * partition p covers [p*S, min((p+1)*S, N)) with S = ceil(N/P); the last one may be short;
