@@ -96,3 +96,27 @@ def test_host_error_prediction_matches_the_oracle(seed):
     eps = float(np.quantile(w, 0.5)) * 0.05
     np.testing.assert_array_equal(pa.predict_fresh(w, d2, r2, G, eps),
                                   O.predict_fresh(w, d2, r2, G, eps))
+
+
+def test_host_prediction_extremes():
+    rng = np.random.default_rng(7)
+    P, G = 12, 3
+    QG = P // G
+    w = rng.dirichlet(np.ones(P), size=QG)
+    d2 = rng.uniform(0.001, 0.01, size=(QG, P))
+    r2 = rng.uniform(0.5, 2.0, size=(QG, P))
+    # a zero bound recomputes everything; an unreachable one only the own groups
+    assert pa.predict_fresh(w, d2, r2, G, 0.0).all()
+    np.testing.assert_array_equal(pa.predict_fresh(w, d2, r2, G, np.inf), np.eye(QG, dtype=np.uint8))
+    # no drift measured (all reference norms zero): only the own groups
+    np.testing.assert_array_equal(pa.predict_fresh(w, d2, np.zeros_like(r2), G, 1e-9),
+                                  np.eye(QG, dtype=np.uint8))
+    # a threshold of zero selects every pair, an unreachable one none
+    assert pa.select_fresh(w, G, 0.0).all()
+    assert not pa.select_fresh(w, G, 2.0).any()
+
+
+def test_binding_rejects_unsupported_dtypes():
+    import torch
+    with pytest.raises(pa.PAError, match="PA_EUNSUPPORTED"):
+        pa._dtype_code(torch.empty(1, dtype=torch.float16))
