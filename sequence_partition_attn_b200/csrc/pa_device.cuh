@@ -179,7 +179,7 @@ __device__ __forceinline__ void tma_prefetch(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
-// 3-D tiled load (no multicast) into shared memory, completing `bar`'s transaction count.
+// 3-D tiled load into this CTA's own shared memory, completing `bar`'s transaction count.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, int x, int y,
                                             int z, uint32_t bar) {
   asm volatile(
