@@ -120,3 +120,22 @@ def test_binding_rejects_unsupported_dtypes():
     import torch
     with pytest.raises(pa.PAError, match="PA_EUNSUPPORTED"):
         pa._dtype_code(torch.empty(1, dtype=torch.float16))
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    # the C ABI compiles as C99 and links against the library; without a GPU the program
+    # checks the device-free calls
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(pa.lib_path())
+    exe = tmp_path / "c_abi_check"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(root, "include"),
+                        os.path.join(root, "tests", "c_abi_check.c"), "-L", libdir, "-lpa",
+                        f"-Wl,-rpath,{libdir}", "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
