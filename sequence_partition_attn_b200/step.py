@@ -251,11 +251,8 @@ def relayout_overlapped(ctx, src_qkv, dst_qkv, n_chunks, part_off, G, o_part, ls
     QG = -(-P // G)
     gpc = per // G                          # groups per chunk
     if milestones is None:
-        milestones, m = [], 1
-        while m < n_chunks:
-            milestones.append(m)
-            m *= 2
-        milestones.append(n_chunks)
+        milestones = chunk_milestones(n_chunks)
+    masks = milestone_masks(QG, gpc, milestones)
     events = []
     for c in range(n_chunks):
         with torch.cuda.stream(s_copy):
@@ -265,13 +262,32 @@ def relayout_overlapped(ctx, src_qkv, dst_qkv, n_chunks, part_off, G, o_part, ls
             ev = torch.cuda.Event()
             ev.record(s_copy)
             events.append(ev)
-    prev = 0
-    for m in milestones:
+    for m, mask in zip(milestones, masks):
         s_attn.wait_event(events[m - 1])
+        pa_partition_attn(ctx, q, k, v, part_off, G, mask, o_part, lse_part, stream=s_attn)
+    return events
+
+
+def chunk_milestones(n_chunks):
+    """Chunk counts after which attention launches: 1, 2, 4, ... and n_chunks."""
+    milestones, m = [], 1
+    while m < n_chunks:
+        milestones.append(m)
+        m *= 2
+    milestones.append(n_chunks)
+    return milestones
+
+
+def milestone_masks(QG, gpc, milestones):
+    """Reuse masks (uint8[QG, QG], 1 = compute) of the attention launches at `milestones`:
+    after chunks [0, m) have moved, every (query group, KV group) pair whose later chunk
+    lies in [previous milestone, m).  Together they select every pair exactly once."""
+    masks, prev = [], 0
+    for m in milestones:
         mask = np.zeros((QG, QG), dtype=np.uint8)
         lo, hi = prev * gpc, m * gpc
         mask[lo:hi, :hi] = 1                # new query chunks x every moved KV chunk
         mask[:lo, lo:hi] = 1                # earlier query chunks x new KV chunks
-        pa_partition_attn(ctx, q, k, v, part_off, G, mask, o_part, lse_part, stream=s_attn)
+        masks.append(mask)
         prev = m
-    return events
+    return masks

@@ -139,3 +139,19 @@ def test_header_is_plain_c_and_links(tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+
+
+@pytest.mark.parametrize("n_chunks,gpc", [(1, 4), (2, 1), (5, 2), (16, 4), (16, 1), (7, 3)])
+def test_overlapped_relayout_launches_cover_every_pair_once(n_chunks, gpc):
+    # the attention launches of the chunked relayout pipeline select every (query group,
+    # KV group) pair exactly once, and only pairs whose chunks have both moved
+    from sequence_partition_attn_b200.step import chunk_milestones, milestone_masks
+    QG = n_chunks * gpc
+    ms = chunk_milestones(n_chunks)
+    assert ms[-1] == n_chunks and ms == sorted(set(ms))
+    masks = milestone_masks(QG, gpc, ms)
+    total = np.sum(masks, axis=0)
+    np.testing.assert_array_equal(total, np.ones((QG, QG)))
+    for m, mask in zip(ms, masks):
+        qg, kg = np.nonzero(mask)
+        assert (qg < m * gpc).all() and (kg < m * gpc).all()
