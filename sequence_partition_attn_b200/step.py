@@ -36,7 +36,7 @@ def attn_flops(part_off, G: int, fresh, B: int, H: int, D: int) -> float:
     return 4.0 * D * B * H * total
 
 
-def merge_bytes(B, H, N, D, P, elem_bytes, with_w=True) -> float:
+def merge_bytes(B, H, N, D, P, elem_bytes) -> float:
     """Algorithmic HBM bytes of the merge: per row P states of (D*elem + 4) read and one
     state written; the importance adds nothing (fused)."""
     row = D * elem_bytes + 4

@@ -155,3 +155,25 @@ def test_overlapped_relayout_launches_cover_every_pair_once(n_chunks, gpc):
     for m, mask in zip(ms, masks):
         qg, kg = np.nonzero(mask)
         assert (qg < m * gpc).all() and (kg < m * gpc).all()
+
+
+def test_algorithmic_work_of_the_configurations():
+    # flop and byte accounting behind every throughput figure, against the counts derived
+    # by hand from the configuration text: 4*D per (query row, valid key) of each fresh
+    # pair; merge bytes P*(D*b + 4) read + (D*b + 4) written per row
+    import workloads as W
+    from sequence_partition_attn_b200.step import attn_flops, merge_bytes
+    expect = {0: (4 * 64 * 2 * 1024 * 1024, None),                        # all pairs fresh
+              1: (4 * 128 * 24 * 512 * 512 * 22, 4096 * 24 * (8 * 260 + 260)),   # 22 of 64 pairs
+              2: (29265744363520, 75600 * 40 * (32 * 260 + 260))}
+    for i, (fl, mb) in expect.items():
+        wl = W.workload(i)
+        assert attn_flops(W.part_offsets(wl.N, wl.P), wl.G, W.reuse_mask(wl), wl.B, wl.H, wl.D) == fl
+        if mb is not None:
+            assert merge_bytes(wl.B, wl.H, wl.N, wl.D, wl.P, wl.elem_bytes) == mb
+    # 720p: 8 query groups of 9452 / 9452 / ... rows with a 9436-row tail (2347 + 3 * 2363)
+    wl = W.workload(2)
+    rows = np.diff(W.group_row_bounds(W.part_offsets(wl.N, wl.P), wl.G))
+    fresh = W.reuse_mask(wl)
+    total = sum(int(rows[q]) * int(rows[k]) for q in range(8) for k in range(8) if fresh[q, k])
+    assert 4 * 128 * 40 * total == 29265744363520
