@@ -14,7 +14,9 @@ oracle's own code.
 * brute force with pure-Python loops and math.exp on tiny inputs;
 * a hand-worked fixture (tests/golden/hand_worked_states.json);
 * the relayout against an index-encoding closed form (SwiftFusion web summary,
-  Methodology 2 "Torus Attention": the chunked all-to-all moves data, nothing else).
+  Methodology 2 "Torus Attention": the chunked all-to-all moves data, nothing else);
+* property-based: the merge against the direct softmax-weighted sum, group splits and
+  the weights' sum on any states drawn by hypothesis, empty ones included.
 """
 import itertools
 import json
@@ -25,6 +27,7 @@ from fractions import Fraction
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 from scipy.special import logsumexp
 
 import oracle as O
@@ -491,3 +494,37 @@ def test_predict_fresh_policy():
     np.testing.assert_array_equal(m, [[1, 0], [0, 1]])
     m = O.predict_fresh(w, d2, r2, 2, eps=0.01)
     np.testing.assert_array_equal(m, [[1, 1], [1, 1]])
+
+
+# --------------------------------------------------------------------------- property-based
+
+
+@settings(max_examples=60, deadline=None)
+@given(P=st.integers(1, 9), R=st.integers(1, 6), seed=st.integers(0, 10_000),
+       n_inf=st.integers(0, 3), split=st.integers(1, 8))
+def test_merge_properties_hold_for_any_states(P, R, seed, n_inf, split):
+    # any states, some of them empty (-inf): the merge equals the direct softmax-weighted
+    # sum, any split into two groups merged separately and then together gives the same,
+    # and the weights exp(LSE_p - LSE) of the non-empty states sum to one per row
+    rng = np.random.default_rng(seed)
+    lse = rng.normal(scale=4.0, size=(P, R))
+    o = rng.standard_normal((P, R, 2))
+    for p in rng.choice(P, size=min(n_inf, P - 1), replace=False):
+        lse[p] = -np.inf
+        o[p] = 0.0
+    mo, ml = O.merge_states(list(o), list(lse))
+    # direct definition, written out independently
+    m = lse.max(axis=0)
+    wts = np.exp(lse - m)
+    ref_l = m + np.log(wts.sum(axis=0))
+    ref_o = (wts[..., None] * o).sum(axis=0) / wts.sum(axis=0)[..., None]
+    np.testing.assert_allclose(ml, ref_l, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(mo, ref_o, rtol=0, atol=1e-12)
+    k = min(split, P)
+    if 0 < k < P:
+        a = O.merge_states(list(o[:k]), list(lse[:k]))
+        b = O.merge_states(list(o[k:]), list(lse[k:]))
+        go, gl = O.merge_states([a[0], b[0]], [a[1], b[1]])
+        np.testing.assert_allclose(gl, ml, atol=1e-12)
+        np.testing.assert_allclose(go, mo, atol=1e-12)
+    np.testing.assert_allclose(np.exp(lse - ml).sum(axis=0), 1.0, atol=1e-12)
