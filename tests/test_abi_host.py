@@ -177,3 +177,13 @@ def test_algorithmic_work_of_the_configurations():
     fresh = W.reuse_mask(wl)
     total = sum(int(rows[q]) * int(rows[k]) for q in range(8) for k in range(8) if fresh[q, k])
     assert 4 * 128 * 40 * total == 29265744363520
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    # no fallback: with libpa.so absent every call raises instead of computing elsewhere
+    monkeypatch.setattr(pa, "_LIB", None)
+    monkeypatch.setattr(pa, "lib_path", lambda: str(tmp_path / "libpa.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        pa.lib()
+    with pytest.raises(RuntimeError, match="missing"):
+        pa.Context(0)
