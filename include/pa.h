@@ -68,6 +68,13 @@
  * would (PA_ECUDA for a launch or runtime error, PA_ETIMEOUT for a device-side wait that
  * gave up).
  *
+ * Fault injection (tests).  PA_INJECT_ENOMEM, a comma-separated list of the sites "init"
+ * (pa_init's status word) and "workspace" (the context workspace), read at each device
+ * allocation, makes those allocations fail with PA_ENOMEM as if cudaMalloc had, without
+ * calling it; the call then behaves as under real memory pressure (pa_init returns no
+ * context; a workspace call returns PA_ENOMEM, launches nothing and leaves the context
+ * usable).
+ *
  * Errors.  Every call returns PA_OK (0) or a negative status; pa_last_error gives a
  * one-line message for the last failure on that context (thread-unsafe per context).
  * Validation happens before anything is enqueued: on error nothing was launched.
@@ -118,6 +125,14 @@ const char* pa_last_error(const pa_ctx* ctx);
 /* Synchronise `stream`, then read and clear the context's device status word.
  * Returns PA_OK, PA_ETIMEOUT if a kernel's bounded wait gave up, or PA_ECUDA. */
 int pa_sync_status(pa_ctx* ctx, void* stream);
+
+/* pa_sync_status with a host-side deadline: poll `stream` (cudaStreamQuery) for up to
+ * timeout_s seconds (0 <= timeout_s <= 86400).  If its work has not finished by then,
+ * return PA_ETIMEOUT without touching the status word -- nothing is cancelled, and the
+ * caller may wait again or tear down; otherwise as pa_sync_status.  The library's
+ * counterpart, on the host, of the bounded device-side waits (the pages describe none).
+ * Errors: PA_EINVAL, PA_ETIMEOUT, PA_ECUDA. */
+int pa_wait_status(pa_ctx* ctx, void* stream, double timeout_s);
 
 /* Library version string. */
 const char* pa_version(void);

@@ -7,7 +7,7 @@ host arrays, and the stream is the current PyTorch CUDA stream unless one is giv
 names follow the C ABI in ``include/pa.h``:
 
     pa_init / Context            pa_partition_attn    pa_merge_states
-    pa_importance                pa_relayout_seq2head pa_sync_status
+    pa_importance                pa_relayout_seq2head pa_sync_status / pa_wait_status
     pa_merge_states_noalloc      pa_compose_states    pa_state_drift
 
 There is no fallback: if ``libpa.so`` is missing or the device is not sm_100 the calls
@@ -32,7 +32,7 @@ PA_F32, PA_BF16 = 0, 1
 PA_MAX_P = 128
 _ERRORS = {-1: "PA_EINVAL", -2: "PA_EALIGN", -3: "PA_EUNSUPPORTED", -4: "PA_ENOMEM",
            -5: "PA_ECUDA", -6: "PA_ETIMEOUT"}
-EXPORTED = ("pa_init", "pa_destroy", "pa_last_error", "pa_sync_status", "pa_version",
+EXPORTED = ("pa_init", "pa_destroy", "pa_last_error", "pa_sync_status", "pa_wait_status", "pa_version",
             "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head",
             "pa_merge_states_noalloc", "pa_compose_states", "pa_state_drift", "pa_selftest_wait")
 
@@ -87,6 +87,7 @@ def lib():
         L.pa_last_error.argtypes = [vp]
         L.pa_last_error.restype = ctypes.c_char_p
         L.pa_sync_status.argtypes = [vp, vp]
+        L.pa_wait_status.argtypes = [vp, vp, ctypes.c_double]
         L.pa_version.restype = ctypes.c_char_p
         L.pa_partition_attn.argtypes = [vp, ctypes.POINTER(_AttnDesc), vp]
         L.pa_merge_states.argtypes = [vp, ctypes.POINTER(_MergeDesc), vp]
@@ -96,7 +97,7 @@ def lib():
         L.pa_relayout_seq2head.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, vp]
         L.pa_state_drift.argtypes = [vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp]
         L.pa_selftest_wait.argtypes = [vp, ctypes.c_double, vp]
-        for f in ("pa_init", "pa_sync_status", "pa_partition_attn", "pa_merge_states", "pa_merge_states_noalloc",
+        for f in ("pa_init", "pa_sync_status", "pa_wait_status", "pa_partition_attn", "pa_merge_states", "pa_merge_states_noalloc",
                   "pa_compose_states", "pa_state_drift", "pa_selftest_wait",
                   "pa_importance", "pa_relayout_seq2head"):
             getattr(L, f).restype = ci
@@ -122,9 +123,14 @@ class Context:
     def ptr(self):
         return self._ptr
 
-    def sync_status(self, stream=None):
-        """pa_sync_status: synchronise the stream, raise if a device wait gave up."""
-        _check(self._ptr, lib().pa_sync_status(self._ptr, _stream(stream)))
+    def sync_status(self, stream=None, timeout=None):
+        """pa_sync_status: synchronise the stream, raise if a device wait gave up.  With
+        `timeout` (seconds), pa_wait_status: raise PAError (PA_ETIMEOUT) if the stream's
+        work has not finished by then (nothing is cancelled)."""
+        if timeout is None:
+            _check(self._ptr, lib().pa_sync_status(self._ptr, _stream(stream)))
+        else:
+            _check(self._ptr, lib().pa_wait_status(self._ptr, _stream(stream), float(timeout)))
 
     def close(self):
         if self._ptr:

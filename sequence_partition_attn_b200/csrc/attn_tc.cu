@@ -33,10 +33,7 @@
 // S_x(j+1) implies PV_x(j) is complete: the softmax may overwrite S_x / P_x columns and
 // touch O_x after waiting only for S_x(j+1).
 //
-// Exponentials: 2^t on full tiles can be split between the MUFU unit and a degree-3
-// polynomial on the FMA pipe (kPolyPairs of every 8 column pairs): Cody-Waite split t = n + f,
-// |f| <= 1/2, 2^f by a minimax polynomial fitted for this kernel (fit_exp2_poly.py, max
-// relative error 7.5e-5), 2^n added to the exponent field.
+// Exponentials run on MUFU (ex2.approx.ftz), one per score.
 #include "pa_device.cuh"
 #include "pa_launch.h"
 
@@ -73,35 +70,6 @@ struct Layout {
 
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;    // move the running max only when it grows by > 8
-// Column pairs out of every 8 whose exponentials run on the FMA pipe (packed polynomial)
-// instead of MUFU, on tiles with every key valid.  Measured at the 720p shape (packed
-// scale/sum in place): 0 -> 1010, 1 -> 998, 2 -> 962, 3 -> 955, 4 -> 921 TFLOP/s, so all
-// exponentials go to MUFU.
-constexpr int kPolyPairs = 0;
-
-// Minimax coefficients of 2^f on [-1/2, 1/2] (relative error), from fit_exp2_poly.py.
-constexpr float kC0 = 0.9999280571937561f;
-constexpr float kC1 = 0.6932609677314758f;
-constexpr float kC2 = 0.24261093139648438f;
-constexpr float kC3 = 0.05517149344086647f;
-
-// 2^t for a pair of values on the FMA pipe, with packed fp32x2 arithmetic (one instruction
-// per pair for the rounding, the reduction and the polynomial).  t is clamped at -126 so
-// that adding n to the exponent field of 2^f (which lies in [0.70, 1.42]) can never
-// underflow the field; n = round(t) lands in the low mantissa bits of t + 1.5 * 2^23.
-__device__ __forceinline__ float2 poly_exp2x2(float2 t) {
-  t.x = fmaxf(t.x, -126.0f);
-  t.y = fmaxf(t.y, -126.0f);
-  const float2 rnd = __fadd2_rn(t, make_float2(12582912.0f, 12582912.0f));
-  const float2 n = __fadd2_rn(rnd, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = __fadd2_rn(t, make_float2(-n.x, -n.y));
-  float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
-  p = __ffma2_rn(p, f, make_float2(kC0, kC0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(rnd.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(rnd.y) << 23)));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -127,7 +95,8 @@ __device__ __forceinline__ float row_max128(const float (&s)[128]) {
 // k1 (shifted back over keys already processed, which the softmax masks), so K and V rows
 // outside the partition are never read: masked keys get P = 0, and 0 * V is 0 only for
 // finite V -- rows of another partition may be non-finite or, in the chunked relayout
-// pipeline, still being written.  Partitions shorter than 128 keys load [k0, k0 + 128).
+// pipeline, still being written.  Partitions shorter than 128 keys load [k0, k0 + 128);
+// the softmax zeroes the V rows past k1 in shared memory before the PV products read them.
 __device__ __forceinline__ int tile_row0(int key, int k0, int k1) {
   return (key + kBN > k1 && k1 - kBN >= k0) ? k1 - kBN : key;
 }
@@ -182,9 +151,9 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint6
 
 // Exponentials of half H of a row (columns 64H .. 64H+63), added to the row-sum chains
 // and packed to bf16 pairs (32 TMEM columns).  Scale-and-shift and the sums use Blackwell's
-// packed fp32x2 FMA / ADD (one instruction per pair).  kFull: every key valid (masked keys
-// hold -inf otherwise, and MUFU's exp2(-inf) = 0 handles them).
-template <bool kFull, int H>
+// packed fp32x2 FMA / ADD (one instruction per pair).  Masked keys hold -inf, and MUFU's
+// exp2(-inf) = 0 handles them, so one copy of the loop serves every tile.
+template <int H>
 __device__ __forceinline__ void exp_pack_half(const float (&s)[128], float m, float sl2, float2 (&acc)[4],
                                               uint32_t (&w)[32]) {
   const float2 scale2 = make_float2(sl2, sl2), neg_m2 = make_float2(-m, -m);
@@ -192,15 +161,7 @@ __device__ __forceinline__ void exp_pack_half(const float (&s)[128], float m, fl
   for (int i = 0; i < 32; ++i) {
     const int c = H * 64 + 2 * i;
     const float2 a = __ffma2_rn(make_float2(s[c], s[c + 1]), scale2, neg_m2);
-    float e0, e1;
-    if (kFull && (i & 7) < kPolyPairs) {
-      const float2 e = poly_exp2x2(a);
-      e0 = e.x;
-      e1 = e.y;
-    } else {
-      e0 = fast_exp2(a.x);
-      e1 = fast_exp2(a.y);
-    }
+    const float e0 = fast_exp2(a.x), e1 = fast_exp2(a.y);
     acc[i & 3] = __fadd2_rn(acc[i & 3], make_float2(e0, e1));
     w[i] = pack_bf16x2(e0, e1);
   }
@@ -468,6 +429,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
           for (int c = 0; c < kBN; ++c) s[c] = (c >= lo && c < lo + nvalid) ? s[c] : -INFINITY;
         }
+        if (x == 0 && nvalid < kBN && tile_row0(key, k0, k1) == key) {
+          // A partition shorter than a tile: the V box runs past the partition end into rows
+          // that may be non-finite (another partition, or rows still being written).  Masked
+          // keys have P = 0, but 0 * inf is NaN in the PV product, so tile a's warps zero
+          // those V rows in shared memory before handing over P (both PV products of this
+          // tile are issued after that hand-off).  A whole 128-byte row of each swizzle atom
+          // is one key, so the swizzle does not matter here.
+          const int st = j % kStages;
+          if (!mbar_wait(bar(L::V_FULL + st), (j / kStages) & 1, abort_flag, status)) { ok = false; break; }
+          if (row >= nvalid) {
+#pragma unroll
+            for (int a = 0; a < L::kAtoms; ++a) {
+              uint4* dst = reinterpret_cast<uint4*>(gbase + L::kV + st * L::kTileBytes + a * kAtomBytes + row * 128);
+#pragma unroll
+              for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+          fence_async_smem();
+        }
         const float mt = row_max128(s) * sl2;
         if (key == k0) {
           // S_x(j) complete implies PV_x(j-1) complete: O_x holds the previous partition.
@@ -498,10 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                          make_float2(0.f, 0.f)};
         {
           uint32_t w[32];
-          // With every exponential on MUFU (kPolyPairs == 0) masked keys need no
-          // separate path: one copy of the loop keeps the hot code small.
-          if (kPolyPairs == 0 || nvalid == kBN) exp_pack_half<true, 0>(s, m, sl2, acc, w);
-          else exp_pack_half<false, 0>(s, m, sl2, acc, w);
+          exp_pack_half<0>(s, m, sl2, acc, w);
           tmem_st32(tS + 0, w);
           tmem_wait_st();
           tc_fence_before();
@@ -509,10 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         {
           uint32_t w[32];
-          // With every exponential on MUFU (kPolyPairs == 0) masked keys need no
-          // separate path: one copy of the loop keeps the hot code small.
-          if (kPolyPairs == 0 || nvalid == kBN) exp_pack_half<true, 1>(s, m, sl2, acc, w);
-          else exp_pack_half<false, 1>(s, m, sl2, acc, w);
+          exp_pack_half<1>(s, m, sl2, acc, w);
           tmem_st32(tS + 32, w);
           tmem_wait_st();
           tc_fence_before();

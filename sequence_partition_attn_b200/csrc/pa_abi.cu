@@ -3,12 +3,14 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <chrono>
 #include <cstdarg>
 #include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <thread>
 
 #include "../../include/pa.h"
 #include "pa_device.cuh"
@@ -119,6 +121,24 @@ int fill_tile_start(pa::AttnTables& t, int tile_rows) {
   return acc;
 }
 
+// Host-side fault injection for tests (no GPU fault involved): PA_INJECT_ENOMEM, a
+// comma-separated list of sites ("init", "workspace"), makes the named device allocations
+// fail as if cudaMalloc had, without calling it.  Read at every allocation, so a process
+// can arm and disarm it between calls.
+bool inject_enomem(const char* site) {
+  const char* env = getenv("PA_INJECT_ENOMEM");
+  if (!env || !*env) return false;
+  const size_t n = strlen(site);
+  for (const char* p = env; *p;) {
+    const char* end = strchr(p, ',');
+    const size_t len = end ? static_cast<size_t>(end - p) : strlen(p);
+    if (len == n && strncmp(p, site, n) == 0) return true;
+    if (!end) break;
+    p = end + 1;
+  }
+  return false;
+}
+
 int check_device(pa_ctx* ctx) {
   int d = -1;
   cudaError_t e = cudaGetDevice(&d);
@@ -135,7 +155,7 @@ int ensure_ws(pa_ctx* ctx, size_t bytes) {
     ctx->ws = nullptr;
     ctx->ws_bytes = 0;
   }
-  if (cudaMalloc(&ctx->ws, bytes) != cudaSuccess) {
+  if (inject_enomem("workspace") || cudaMalloc(&ctx->ws, bytes) != cudaSuccess) {
     cudaGetLastError();
     ctx->ws = nullptr;
     return fail(ctx, PA_ENOMEM, "workspace allocation of %zu bytes failed", bytes);
@@ -171,10 +191,10 @@ int fill_blk_start(const pa::AttnTables& t, int* blk_start) {
 }
 
 int launch_reduce(pa_ctx* ctx, const pa::AttnTables& t, const int* blk_start, int blocks_per_bh, int BH,
-                  float* w, cudaStream_t st) {
+                  const float* w_partial, float* w, cudaStream_t st) {
   pa::ReduceWParams r;
   memset(&r, 0, sizeof r);
-  r.w_partial = static_cast<const float*>(ctx->ws);
+  r.w_partial = w_partial;
   r.w = w;
   r.BH = BH;
   r.P = t.P;
@@ -187,6 +207,67 @@ int launch_reduce(pa_ctx* ctx, const pa::AttnTables& t, const int* blk_start, in
   }
   int e = pa::launch_reduce_w(r, st);
   return e ? cuda_fail(ctx, e, "reduce_w launch") : PA_OK;
+}
+
+// Argument checks and kernel parameters shared by pa_merge_states and
+// pa_merge_states_noalloc: everything but the importance scratch (prm.w_partial stays
+// null).  Errors are recorded on ctx (or, with ctx == NULL, in the thread's init-error
+// slot that pa_last_error(NULL) reads).  *n_partials is the number of per-block importance
+// sums the fused importance needs (0 without w); *launch is false when there is nothing to
+// launch (N == 0).
+int prepare_merge(pa_ctx* ctx, const pa_merge_desc* d, pa::AttnTables& t, pa::MergeParams& prm,
+                  size_t* n_partials, bool* launch) {
+  *launch = false;
+  *n_partials = 0;
+  if (!d) return fail(ctx, PA_EINVAL, "desc is NULL");
+  if (d->dtype != PA_BF16 && d->dtype != PA_F32) return fail(ctx, PA_EUNSUPPORTED, "dtype %d", (int)d->dtype);
+  if (d->D != 64 && d->D != 128) return fail(ctx, PA_EUNSUPPORTED, "D=%d (supported: 64, 128)", d->D);
+  if (d->B < 1 || d->H < 1 || d->N < 0) return fail(ctx, PA_EINVAL, "B=%d H=%d N=%d", d->B, d->H, d->N);
+  const long long BH = static_cast<long long>(d->B) * d->H;
+  if (BH > 0x7fffffffLL) return fail(ctx, PA_EINVAL, "B*H too large");
+  int rc = build_tables(ctx, d->N, d->P, d->G, d->part_off, d->fresh, t);
+  if (rc) return rc;
+  bool all_fresh = true;
+  for (int qg = 0; qg < t.QG; ++qg)
+    for (int p = 0; p < t.P; ++p) all_fresh &= pa::fresh_bit(t.fresh_bits, qg, p);
+  if (d->N == 0) return PA_OK;
+  if (!d->o_fresh || !d->lse_fresh || !d->o || !d->lse) return fail(ctx, PA_EINVAL, "null tensor pointer");
+  if (!all_fresh && (!d->o_cached || !d->lse_cached))
+    return fail(ctx, PA_EINVAL, "cached states are NULL but the mask reuses some pairs");
+  if (d->cached_per_group != 0 && d->cached_per_group != 1)
+    return fail(ctx, PA_EINVAL, "cached_per_group=%d (0 or 1)", d->cached_per_group);
+  if (d->cached_per_group && d->w)
+    return fail(ctx, PA_EINVAL, "importance needs per-partition cached states (w must be NULL with cached_per_group)");
+  if (!aligned(d->o_fresh, 16) || !aligned(d->o, 16) || (d->o_cached && !aligned(d->o_cached, 16)))
+    return fail(ctx, PA_EALIGN, "o_fresh, o_cached and o must be 16-byte aligned");
+  if (!aligned(d->lse_fresh, 4) || !aligned(d->lse, 4) || (d->lse_cached && !aligned(d->lse_cached, 4)) ||
+      (d->w && !aligned(d->w, 4)))
+    return fail(ctx, PA_EALIGN, "lse arrays and w must be 4-byte aligned");
+  memset(&prm, 0, sizeof prm);
+  const int bpb = fill_blk_start(t, prm.blk_start);
+  const long long blocks = BH * bpb;
+  if (blocks > 0x7fffffffLL) return fail(ctx, PA_EINVAL, "too many row blocks");
+  prm.o_fresh = d->o_fresh;
+  prm.lse_fresh = d->lse_fresh;
+  prm.o_cached = d->o_cached;
+  prm.lse_cached = d->lse_cached;
+  prm.o = d->o;
+  prm.lse = d->lse;
+  prm.w_partial = nullptr;
+  prm.BH = (int)BH;
+  prm.N = d->N;
+  prm.D = d->D;
+  prm.P = t.P;
+  prm.G = t.G;
+  prm.QG = t.QG;
+  prm.blocks_per_bh = bpb;
+  prm.cached_per_group = d->cached_per_group;
+  memcpy(prm.part_off, t.part_off, sizeof prm.part_off);
+  memcpy(prm.qg_row0, t.qg_row0, sizeof prm.qg_row0);
+  memcpy(prm.fresh_bits, t.fresh_bits, sizeof prm.fresh_bits);
+  if (d->w) *n_partials = static_cast<size_t>(blocks) * t.P;
+  *launch = true;
+  return PA_OK;
 }
 
 }  // namespace
@@ -218,7 +299,8 @@ int pa_init(int device, pa_ctx** out) {
   ctx->sm_count = prop.multiProcessorCount;
   const char* dbg = getenv("PA_DEBUG");
   ctx->debug = dbg && *dbg && strcmp(dbg, "0") != 0;
-  if (cudaMalloc(&ctx->d_status, sizeof(int)) != cudaSuccess || cudaMemset(ctx->d_status, 0, sizeof(int)) != cudaSuccess) {
+  if (inject_enomem("init") || cudaMalloc(&ctx->d_status, sizeof(int)) != cudaSuccess ||
+      cudaMemset(ctx->d_status, 0, sizeof(int)) != cudaSuccess) {
     cudaGetLastError();
     if (ctx->d_status) cudaFree(ctx->d_status);
     delete ctx;
@@ -237,18 +319,44 @@ void pa_destroy(pa_ctx* ctx) {
 
 const char* pa_last_error(const pa_ctx* ctx) { return ctx ? ctx->err.c_str() : g_init_err.c_str(); }
 
-int pa_sync_status(pa_ctx* ctx, void* stream) {
-  if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
-  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaStreamSynchronize");
+// Read and clear the context's status word once the stream's work is complete.
+static int read_status(pa_ctx* ctx) {
   int h = 0;
-  e = cudaMemcpy(&h, ctx->d_status, sizeof(int), cudaMemcpyDeviceToHost);
+  cudaError_t e = cudaMemcpy(&h, ctx->d_status, sizeof(int), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "status read");
   if (h != 0) {
     cudaMemset(ctx->d_status, 0, sizeof(int));
     return fail(ctx, PA_ETIMEOUT, "a device-side wait gave up (status %d)", h);
   }
   return PA_OK;
+}
+
+int pa_sync_status(pa_ctx* ctx, void* stream) {
+  if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaStreamSynchronize");
+  return read_status(ctx);
+}
+
+int pa_wait_status(pa_ctx* ctx, void* stream, double timeout_s) {
+  if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
+  if (!(timeout_s >= 0.0) || timeout_s > 86400.0)
+    return fail(ctx, PA_EINVAL, "timeout_s=%g outside [0, 86400]", timeout_s);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto t0 = std::chrono::steady_clock::now();
+  const auto limit = std::chrono::duration<double>(timeout_s);
+  auto nap = std::chrono::microseconds(20);
+  while (true) {
+    cudaError_t e = cudaStreamQuery(st);
+    if (e == cudaSuccess) break;
+    if (e != cudaErrorNotReady) return cuda_fail(ctx, e, "cudaStreamQuery");
+    if (std::chrono::steady_clock::now() - t0 >= limit)
+      return fail(ctx, PA_ETIMEOUT, "the stream's work did not finish within %g s (host deadline); "
+                  "it was not cancelled and may be waited for again", timeout_s);
+    std::this_thread::sleep_for(nap);
+    if (nap < std::chrono::microseconds(2000)) nap *= 2;
+  }
+  return read_status(ctx);
 }
 
 static int pa_partition_attn_impl(pa_ctx* ctx, const pa_attn_desc* d, void* stream) {
@@ -317,64 +425,21 @@ static int pa_partition_attn_impl(pa_ctx* ctx, const pa_attn_desc* d, void* stre
 
 static int pa_merge_states_impl(pa_ctx* ctx, const pa_merge_desc* d, void* stream) {
   if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
-  if (!d) return fail(ctx, PA_EINVAL, "desc is NULL");
-  if (d->dtype != PA_BF16 && d->dtype != PA_F32) return fail(ctx, PA_EUNSUPPORTED, "dtype %d", (int)d->dtype);
-  if (d->D != 64 && d->D != 128) return fail(ctx, PA_EUNSUPPORTED, "D=%d (supported: 64, 128)", d->D);
-  if (d->B < 1 || d->H < 1 || d->N < 0) return fail(ctx, PA_EINVAL, "B=%d H=%d N=%d", d->B, d->H, d->N);
-  const long long BH = static_cast<long long>(d->B) * d->H;
   pa::AttnTables t;
-  int rc = build_tables(ctx, d->N, d->P, d->G, d->part_off, d->fresh, t);
-  if (rc) return rc;
-  bool all_fresh = true;
-  for (int qg = 0; qg < t.QG; ++qg)
-    for (int p = 0; p < t.P; ++p) all_fresh &= pa::fresh_bit(t.fresh_bits, qg, p);
-  if (d->N == 0) {
-    return PA_OK;
-  }
-  if (!d->o_fresh || !d->lse_fresh || !d->o || !d->lse) return fail(ctx, PA_EINVAL, "null tensor pointer");
-  if (!all_fresh && (!d->o_cached || !d->lse_cached))
-    return fail(ctx, PA_EINVAL, "cached states are NULL but the mask reuses some pairs");
-  if (d->cached_per_group != 0 && d->cached_per_group != 1)
-    return fail(ctx, PA_EINVAL, "cached_per_group=%d (0 or 1)", d->cached_per_group);
-  if (d->cached_per_group && d->w)
-    return fail(ctx, PA_EINVAL, "importance needs per-partition cached states (w must be NULL with cached_per_group)");
-  if (!aligned(d->o_fresh, 16) || !aligned(d->o, 16) || (d->o_cached && !aligned(d->o_cached, 16)))
-    return fail(ctx, PA_EALIGN, "o_fresh, o_cached and o must be 16-byte aligned");
-  if (!aligned(d->lse_fresh, 4) || !aligned(d->lse, 4) || (d->lse_cached && !aligned(d->lse_cached, 4)) ||
-      (d->w && !aligned(d->w, 4)))
-    return fail(ctx, PA_EALIGN, "lse arrays and w must be 4-byte aligned");
+  pa::MergeParams prm;
+  size_t n_partials = 0;
+  bool launch = false;
+  int rc = prepare_merge(ctx, d, t, prm, &n_partials, &launch);
+  if (rc || !launch) return rc;
   if ((rc = check_device(ctx))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-
-  pa::MergeParams prm;
-  memset(&prm, 0, sizeof prm);
-  const int bpb = fill_blk_start(t, prm.blk_start);
-  const long long blocks = BH * bpb;
-  if (blocks > 0x7fffffffLL) return fail(ctx, PA_EINVAL, "too many row blocks");
   if (d->w) {
-    if ((rc = ensure_ws(ctx, static_cast<size_t>(blocks) * t.P * sizeof(float)))) return rc;
+    if ((rc = ensure_ws(ctx, n_partials * sizeof(float)))) return rc;
+    prm.w_partial = static_cast<float*>(ctx->ws);
   }
-  prm.o_fresh = d->o_fresh;
-  prm.lse_fresh = d->lse_fresh;
-  prm.o_cached = d->o_cached;
-  prm.lse_cached = d->lse_cached;
-  prm.o = d->o;
-  prm.lse = d->lse;
-  prm.w_partial = d->w ? static_cast<float*>(ctx->ws) : nullptr;
-  prm.BH = (int)BH;
-  prm.N = d->N;
-  prm.D = d->D;
-  prm.P = t.P;
-  prm.G = t.G;
-  prm.QG = t.QG;
-  prm.blocks_per_bh = bpb;
-  prm.cached_per_group = d->cached_per_group;
-  memcpy(prm.part_off, t.part_off, sizeof prm.part_off);
-  memcpy(prm.qg_row0, t.qg_row0, sizeof prm.qg_row0);
-  memcpy(prm.fresh_bits, t.fresh_bits, sizeof prm.fresh_bits);
   int e = pa::launch_merge(prm, d->dtype, st);
   if (e) return cuda_fail(ctx, e, "merge launch");
-  if (d->w) return launch_reduce(ctx, t, prm.blk_start, bpb, (int)BH, d->w, st);
+  if (d->w) return launch_reduce(ctx, t, prm.blk_start, prm.blocks_per_bh, prm.BH, prm.w_partial, d->w, st);
   return PA_OK;
 }
 
@@ -446,7 +511,7 @@ static int pa_importance_impl(pa_ctx* ctx, int B, int H, int N, int P, int G, co
     int e = pa::launch_importance(prm, st);
     if (e) return cuda_fail(ctx, e, "importance launch");
   }
-  return launch_reduce(ctx, t, prm.blk_start, bpb, (int)BH, w, st);
+  return launch_reduce(ctx, t, prm.blk_start, bpb, (int)BH, static_cast<const float*>(ctx->ws), w, st);
 }
 
 static int pa_state_drift_impl(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int P, int G,
@@ -624,84 +689,28 @@ int noalloc_scratch(int device, float** out) {
 }  // namespace
 
 extern "C" int pa_merge_states_noalloc(const pa_merge_desc* d, void* stream) {
-  if (!d) return fail(nullptr, PA_EINVAL, "desc is NULL");
-  if (d->dtype != PA_BF16 && d->dtype != PA_F32) return fail(nullptr, PA_EUNSUPPORTED, "dtype %d", (int)d->dtype);
-  if (d->D != 64 && d->D != 128) return fail(nullptr, PA_EUNSUPPORTED, "D=%d (supported: 64, 128)", d->D);
-  if (d->B < 1 || d->H < 1 || d->N < 0) return fail(nullptr, PA_EINVAL, "B=%d H=%d N=%d", d->B, d->H, d->N);
-  const long long BH = static_cast<long long>(d->B) * d->H;
   pa::AttnTables t;
-  int rc = build_tables(nullptr, d->N, d->P, d->G, d->part_off, d->fresh, t);
-  if (rc) return rc;
-  bool all_fresh = true;
-  for (int qg = 0; qg < t.QG; ++qg)
-    for (int p = 0; p < t.P; ++p) all_fresh &= pa::fresh_bit(t.fresh_bits, qg, p);
-  if (d->N == 0) return PA_OK;
-  if (!d->o_fresh || !d->lse_fresh || !d->o || !d->lse) return fail(nullptr, PA_EINVAL, "null tensor pointer");
-  if (!all_fresh && (!d->o_cached || !d->lse_cached))
-    return fail(nullptr, PA_EINVAL, "cached states are NULL but the mask reuses some pairs");
-  if (d->cached_per_group != 0 && d->cached_per_group != 1)
-    return fail(nullptr, PA_EINVAL, "cached_per_group=%d (0 or 1)", d->cached_per_group);
-  if (d->cached_per_group && d->w)
-    return fail(nullptr, PA_EINVAL, "importance needs per-partition cached states (w must be NULL with cached_per_group)");
-  if (!aligned(d->o_fresh, 16) || !aligned(d->o, 16) || (d->o_cached && !aligned(d->o_cached, 16)))
-    return fail(nullptr, PA_EALIGN, "o_fresh, o_cached and o must be 16-byte aligned");
-  if (!aligned(d->lse_fresh, 4) || !aligned(d->lse, 4) || (d->lse_cached && !aligned(d->lse_cached, 4)) ||
-      (d->w && !aligned(d->w, 4)))
-    return fail(nullptr, PA_EALIGN, "lse arrays and w must be 4-byte aligned");
   pa::MergeParams prm;
-  memset(&prm, 0, sizeof prm);
-  const int bpb = fill_blk_start(t, prm.blk_start);
-  const long long blocks = BH * bpb;
-  if (blocks > 0x7fffffffLL) return fail(nullptr, PA_EINVAL, "too many row blocks");
+  size_t n_partials = 0;
+  bool launch = false;
+  int rc = prepare_merge(nullptr, d, t, prm, &n_partials, &launch);
+  if (rc || !launch) return rc;
   float* scratch = nullptr;
   if (d->w) {
-    const unsigned long long need = static_cast<unsigned long long>(blocks) * t.P;
-    if (need > kNoAllocScratchFloats)
+    if (n_partials > kNoAllocScratchFloats)
       return fail(nullptr, PA_EINVAL,
-                  "importance scratch of %llu floats exceeds the fixed %zu (B*H*ceil(rows/128 per query "
+                  "importance scratch of %zu floats exceeds the fixed %zu (B*H*ceil(rows/128 per query "
                   "group)*P); use pa_merge_states",
-                  need, kNoAllocScratchFloats);
+                  n_partials, kNoAllocScratchFloats);
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(nullptr, PA_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
     if ((rc = noalloc_scratch(dev, &scratch))) return rc;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  prm.o_fresh = d->o_fresh;
-  prm.lse_fresh = d->lse_fresh;
-  prm.o_cached = d->o_cached;
-  prm.lse_cached = d->lse_cached;
-  prm.o = d->o;
-  prm.lse = d->lse;
   prm.w_partial = scratch;
-  prm.BH = (int)BH;
-  prm.N = d->N;
-  prm.D = d->D;
-  prm.P = t.P;
-  prm.G = t.G;
-  prm.QG = t.QG;
-  prm.blocks_per_bh = bpb;
-  prm.cached_per_group = d->cached_per_group;
-  memcpy(prm.part_off, t.part_off, sizeof prm.part_off);
-  memcpy(prm.qg_row0, t.qg_row0, sizeof prm.qg_row0);
-  memcpy(prm.fresh_bits, t.fresh_bits, sizeof prm.fresh_bits);
   int e = pa::launch_merge(prm, d->dtype, st);
   if (e) return fail(nullptr, PA_ECUDA, "merge launch: %s", cudaGetErrorString(static_cast<cudaError_t>(e)));
   if (!d->w) return PA_OK;
-  pa::ReduceWParams r;
-  memset(&r, 0, sizeof r);
-  r.w_partial = scratch;
-  r.w = d->w;
-  r.BH = (int)BH;
-  r.P = t.P;
-  r.QG = t.QG;
-  r.blocks_per_bh = bpb;
-  for (int g = 0; g <= t.QG; ++g) r.blk_start[g] = prm.blk_start[g];
-  for (int g = 0; g < t.QG; ++g) {
-    const long long rows = t.qg_row0[g + 1] - t.qg_row0[g];
-    r.inv_count[g] = rows > 0 ? 1.0 / (static_cast<double>(rows) * BH) : 0.0;
-  }
-  e = pa::launch_reduce_w(r, st);
-  if (e) return fail(nullptr, PA_ECUDA, "reduce_w launch: %s", cudaGetErrorString(static_cast<cudaError_t>(e)));
-  return PA_OK;
+  return launch_reduce(nullptr, t, prm.blk_start, prm.blocks_per_bh, prm.BH, scratch, d->w, st);
 }

@@ -222,6 +222,9 @@ class Trajectory:
                               self.cache_lse, stream=stream)
             pa_merge_states(self.ctx, self.part_off, self.G, None, self.cache_o, self.cache_lse,
                             None, None, self.o, self.lse, self.w, stream=stream)
+            # the merge runs on `stream`, which need not be torch's current stream: wait for
+            # it (and check its bounded waits) before the host reads w
+            self.ctx.sync_status(stream)
             self.w_stored = self.w.cpu().numpy().astype(np.float64)
             return mask
         mask = self._mask(q, k, v, stream)
@@ -243,11 +246,11 @@ def relayout_overlapped(ctx, src_qkv, dst_qkv, n_chunks, part_off, G, o_part, ls
     attention launch early and the number of partially filled launches small.  Chunk
     boundaries must be group boundaries.  Returns the relayout events.
     """
+    check_chunk_bounds(part_off, G, n_chunks)
     src_q, src_k, src_v = src_qkv
     q, k, v = dst_qkv
     P = len(part_off) - 1
     per = P // n_chunks
-    assert per * n_chunks == P and per % G == 0
     QG = -(-P // G)
     gpc = per // G                          # groups per chunk
     if milestones is None:
@@ -266,6 +269,28 @@ def relayout_overlapped(ctx, src_qkv, dst_qkv, n_chunks, part_off, G, o_part, ls
         s_attn.wait_event(events[m - 1])
         pa_partition_attn(ctx, q, k, v, part_off, G, mask, o_part, lse_part, stream=s_attn)
     return events
+
+
+def check_chunk_bounds(part_off, G: int, n_chunks: int) -> None:
+    """Raise ValueError unless every relayout chunk ends on a group boundary.
+
+    pa_relayout_seq2head cuts the sequence at multiples of ceil(N / n_chunks); attention
+    after chunk c covers the partitions [0, c * P / n_chunks), i.e. the tokens
+    [0, part_off[c * P / n_chunks]).  The two must coincide, or attention reads K/V rows
+    that the other stream has not moved yet."""
+    off = np.asarray(part_off, dtype=np.int64)
+    P = len(off) - 1
+    N = int(off[-1])
+    if n_chunks < 1 or P % n_chunks:
+        raise ValueError(f"P={P} partitions do not split into {n_chunks} chunks")
+    per = P // n_chunks
+    if per % G:
+        raise ValueError(f"a chunk of {per} partitions is not a whole number of groups of {G}")
+    step = -(-N // n_chunks)
+    for c in range(n_chunks + 1):
+        if int(off[c * per]) != min(c * step, N):
+            raise ValueError(f"chunk {c} boundary: relayout at token {min(c * step, N)}, "
+                             f"partitions at token {int(off[c * per])}")
 
 
 def chunk_milestones(n_chunks):

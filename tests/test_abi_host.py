@@ -157,6 +157,30 @@ def test_overlapped_relayout_launches_cover_every_pair_once(n_chunks, gpc):
         assert (qg < m * gpc).all() and (kg < m * gpc).all()
 
 
+@pytest.mark.parametrize("N,P,G,n_chunks,ok", [
+    (115200, 64, 1, 16, True),      # the Ulysses layout workload: 7200-token chunks
+    (100, 8, 1, 4, False),          # chunks end at 25/50/75, partitions at 26/52/78
+    (96, 8, 2, 4, True),
+    (96, 8, 4, 4, False),           # 2 partitions per chunk, groups of 4
+    (96, 8, 1, 3, False),           # 8 partitions do not split into 3 chunks
+    (75600, 32, 4, 8, False),       # the 720p partitioning (S = 2363) against 9450-token chunks
+])
+def test_overlapped_relayout_rejects_chunks_off_the_partition_bounds(N, P, G, n_chunks, ok):
+    # the chunked pipeline starts attention on partitions whose K/V rows the relayout has
+    # moved: chunk and partition boundaries must coincide, or it raises before any launch
+    import workloads as W
+    from sequence_partition_attn_b200.step import check_chunk_bounds, relayout_overlapped
+    off = W.part_offsets(N, P)
+    if ok:
+        check_chunk_bounds(off, G, n_chunks)
+    else:
+        with pytest.raises(ValueError):
+            check_chunk_bounds(off, G, n_chunks)
+        with pytest.raises(ValueError):      # raised before the first CUDA call
+            relayout_overlapped(None, (None,) * 3, (None,) * 3, n_chunks, off, G, None, None,
+                                None, None)
+
+
 def test_algorithmic_work_of_the_configurations():
     # flop and byte accounting behind every throughput figure, against the counts derived
     # by hand from the configuration text: 4*D per (query row, valid key) of each fresh

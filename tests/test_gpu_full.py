@@ -1,7 +1,8 @@
 """Full-size GPU parity: the 720p step in the launch configuration bench.py times, the
 10-step denoising trajectory with anchor steps, and the Ulysses-layout workload with the
 chunked relayout overlapped with attention.  Sampled outputs are compared with the fp64
-oracle row by row; w at full size is checked through properties that hold at any size and
+oracle row by row; w at full size is the oracle's fp64 importance reduction over every row
+of the states the merge took, checked as well through properties that hold at any size and
 against the stand-alone importance call."""
 import numpy as np
 import pytest
@@ -72,7 +73,16 @@ def test_720p_step_full_size_sampled_rows(pa):
     assert np.all(w >= 0)
     np.testing.assert_allclose(w.sum(axis=1), 1.0, atol=1e-3)
     assert maxerr(w, w2.cpu().numpy()) <= 1e-5
-    del step, chosen
+    # the full-size importance reduction (every row of every query group, all heads) done
+    # by the oracle in fp64 on the states the merge took; those states are checked against
+    # the oracle's own, computed from Q, K, V, on the sampled rows below
+    chosen_h = chosen.cpu().numpy().astype(np.float64)
+    lse_h = step.lse.cpu().numpy().astype(np.float64)
+    del chosen
+    rw = O.importance(chosen_h, lse_h, off, wl.G)
+    del chosen_h, lse_h
+    assert maxerr(w, rw) <= TOL["bf16"]["w"], maxerr(w, rw)
+    del step
     torch.cuda.empty_cache()
 
     ones = np.ones_like(fresh)
@@ -101,7 +111,7 @@ def test_720p_step_full_size_sampled_rows(pa):
     ctx.close()
 
 
-def _run_trajectory(pa, wl, quality_heads=0, policy="threshold", margin=0.15):
+def _run_trajectory(pa, wl, quality_heads=0, policy="threshold", margin=0.15, side_stream=False):
     from sequence_partition_attn_b200.step import Trajectory
     off = W.part_offsets(wl.N, wl.P)
     host = W.make_qkv(wl)
@@ -120,7 +130,15 @@ def _run_trajectory(pa, wl, quality_heads=0, policy="threshold", margin=0.15):
     for s in range(wl.steps):
         if s > 0:
             k, v = W.drift_kv(wl, k, v, s)
-        mask = traj.step(s, qd, k.to(DEV), v.to(DEV))          # mask from the GPU's stored w
+        kd, vd = k.to(DEV), v.to(DEV)
+        if side_stream:
+            # the step runs on a stream that is not torch's current one
+            side = torch.cuda.Stream(device=DEV)
+            side.wait_stream(torch.cuda.current_stream())
+            mask = traj.step(s, qd, kd, vd, stream=side)
+            ctx.sync_status(side)
+        else:
+            mask = traj.step(s, qd, kd, vd)                       # mask from the GPU's stored w
         ctx.sync_status()
         o = traj.o.float().cpu().numpy()
         lse = traj.lse.cpu().numpy()
@@ -181,6 +199,15 @@ def test_denoising_trajectory_with_reuse(pa):
     report = _run_trajectory(pa, wl, quality_heads=4)
     assert report[0][1] == wl.QG * wl.KG and report[5][1] == wl.QG * wl.KG
     assert any(r[1] < wl.QG * wl.KG for r in report)           # reuse happened
+
+
+def test_denoising_trajectory_on_a_side_stream(pa):
+    # every launch of the trajectory on a stream other than torch's current one: the host
+    # must still read the anchor's importance only after the merge that writes it
+    base = W.workload(3)
+    wl = W.small_variant(base, grid=base.grid, H=4, threshold=0.12)
+    report = _run_trajectory(pa, wl, side_stream=True)
+    assert any(r[1] < wl.QG * wl.KG for r in report)
 
 
 def test_denoising_trajectory_online_prediction(pa):

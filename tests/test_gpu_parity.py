@@ -248,28 +248,40 @@ def test_empty_sequence_is_a_no_op(pa, ctx):
     ctx.sync_status()
 
 
-def test_partition_state_reads_no_other_partition(pa, ctx):
-    # A partition of >= 128 keys must not depend on K/V rows of any other partition, even
-    # non-finite ones (its last partial tile is loaded ending at the partition end).
-    wl = W.small_variant(W.workload(1), grid=(1, 25, 40), H=2, P=4, G=1, mask="all")   # 250 keys each
+@pytest.mark.parametrize("grid,P,p_sel", [((1, 25, 40), 4, 1),      # 250 keys: shifted last tile
+                                          ((1, 32, 64), 128, 5),    # 16 keys: shorter than a tile
+                                          ((1, 20, 23), 8, 7)])     # 54 keys, last partition
+def test_partition_state_reads_no_other_partition(pa, ctx, grid, P, p_sel):
+    # A partition's state must not depend on K/V rows of any other partition, even
+    # non-finite ones: a partial last tile of a partition of >= 128 keys is loaded ending at
+    # the partition end, and for a partition shorter than a tile the V rows past its end
+    # are zeroed in shared memory before the PV product reads them.
+    wl = W.small_variant(W.workload(1), grid=grid, H=2, P=P, G=1, mask="all")
     t = W.make_qkv(wl)
     off = W.part_offsets(wl.N, wl.P)
     q, k, v = (t[n].to(DEV) for n in ("q", "k", "v"))
-    fresh = np.zeros((4, 4), dtype=np.uint8)
-    fresh[:, 1] = 1                                              # every query group x partition 1
-    o1 = torch.zeros(4, 1, 2, wl.N, 128, dtype=torch.bfloat16, device=DEV)
-    l1 = torch.zeros(4, 1, 2, wl.N, device=DEV)
+    fresh = np.zeros((P, P), dtype=np.uint8)
+    fresh[:, p_sel] = 1                                          # every query group x one partition
+    o1 = torch.zeros(P, 1, 2, wl.N, 128, dtype=torch.bfloat16, device=DEV)
+    l1 = torch.zeros(P, 1, 2, wl.N, device=DEV)
     pa.pa_partition_attn(ctx, q, k, v, off, 1, fresh, o1, l1)
     k2, v2 = k.clone(), v.clone()
-    for p in (0, 2, 3):
-        k2[:, :, off[p]:off[p + 1]] = float("nan")
-        v2[:, :, off[p]:off[p + 1]] = float("inf")
+    for p in range(P):
+        if p != p_sel:
+            k2[:, :, off[p]:off[p + 1]] = float("nan")
+            v2[:, :, off[p]:off[p + 1]] = float("inf")
     o2 = torch.zeros_like(o1)
     l2 = torch.zeros_like(l1)
     pa.pa_partition_attn(ctx, q, k2, v2, off, 1, fresh, o2, l2)
     ctx.sync_status()
-    assert torch.isfinite(o2[1].float()).all() and torch.isfinite(l2[1]).all()
-    assert torch.equal(o1[1].view(torch.int16), o2[1].view(torch.int16)) and torch.equal(l1[1], l2[1])
+    assert torch.isfinite(o2[p_sel].float()).all() and torch.isfinite(l2[p_sel]).all()
+    assert torch.equal(o1[p_sel].view(torch.int16), o2[p_sel].view(torch.int16))
+    assert torch.equal(l1[p_sel], l2[p_sel])
+    # and the clean run matches the oracle on that partition
+    qf, kf, vf = (W.to_f64(t[n]) for n in ("q", "k", "v"))
+    ro, rl, _ = O.partition_states(qf, kf, vf, off, 1, fresh, wl.scale)
+    assert maxerr(o1[p_sel].float().cpu().numpy(), ro[p_sel]) <= TOL["bf16"]["o"]
+    assert maxerr(l1[p_sel].cpu().numpy(), rl[p_sel]) <= TOL["bf16"]["lse"]
 
 
 # --------------------------------------------------------------------------- group compose
@@ -330,7 +342,7 @@ def test_merge_with_composed_cache_against_oracle(pa, ctx):
 
 def test_merge_with_composed_cache(pa, ctx):
     # 720p recipe on a reduced grid, states from the attention kernel: the composed-cache
-    # merge agrees with the per-partition merge (GPU against GPU: associativity).
+    # merge agrees with the per-partition merge (associativity) and with the oracle.
     wl = W.small_variant(W.workload(2), grid=(3, 45, 80), H=2)
     t = W.make_qkv(wl)
     kc, vc = W.make_cached_kv(wl, t["k"], t["v"])
@@ -354,6 +366,21 @@ def test_merge_with_composed_cache(pa, ctx):
     ctx.sync_status()
     assert maxerr(o1.float().cpu().numpy(), o2.float().cpu().numpy()) <= TOL["bf16"]["o"]
     assert maxerr(l1.cpu().numpy(), l2.cpu().numpy()) <= 1e-5
+    # and against the oracle from Q, K, V on sampled rows (every group boundary included):
+    # fresh and cached states, composition of the cache per KV group, merge
+    gb = W.group_row_bounds(off, wl.G)
+    rng = np.random.default_rng(21)
+    rows = np.unique(np.concatenate([rng.choice(N, 160, replace=False), gb[1:-1], gb[1:-1] - 1,
+                                     np.arange(N - 8, N)]))
+    ones = np.ones_like(fresh)
+    qf, kf, vf = (W.to_f64(t[n]) for n in ("q", "k", "v"))
+    rof, rlf, _ = O.partition_states(qf, kf, vf, off, wl.G, fresh, wl.scale, rows=rows)
+    roc, rlc, _ = O.partition_states(qf, W.to_f64(kc), W.to_f64(vc), off, wl.G, ones, wl.scale, rows=rows)
+    rco, rcl = O.compose_states(roc, rlc, wl.G)
+    ro, rl = O.merge_with_composed_cache(rof, rlf, rco, rcl, off, wl.G, fresh, rows=rows)
+    ri = torch.as_tensor(rows, device=DEV)
+    assert maxerr(o1.index_select(2, ri).float().cpu().numpy(), ro) <= TOL["bf16"]["o"]
+    assert maxerr(l1.index_select(2, ri).cpu().numpy(), rl) <= TOL["bf16"]["lse"]
     w = torch.empty(wl.QG, P, device=DEV)
     with pytest.raises(pa.PAError, match="PA_EINVAL"):
         pa.pa_merge_states(ctx, off, wl.G, fresh, of, lf, ocg, lcg, o1, l1, w, cached_per_group=True)
@@ -477,5 +504,61 @@ def test_debug_mode_reports_at_the_call(pa, monkeypatch):
         dst = torch.empty(2, 64, 64, dtype=torch.bfloat16, device=DEV)
         pa.pa_relayout_seq2head(c, src, dst)             # an ordinary call passes through
         assert torch.equal(dst.cpu(), src.cpu().transpose(0, 1))
+    finally:
+        c.close()
+
+
+def test_host_deadline_leaves_the_stream_running_and_the_context_usable(pa, ctx):
+    # pa_wait_status gives up on the host after its deadline while a kernel still waits
+    # (its own device-side limit is longer); nothing is cancelled: a later wait sees the
+    # kernel finish and the device-side give-up it recorded, and the context keeps working
+    import time
+    pa.pa_selftest_wait(ctx, 1.0)
+    t0 = time.time()
+    with pytest.raises(pa.PAError, match="PA_ETIMEOUT.*host deadline"):
+        ctx.sync_status(timeout=0.05)
+    assert time.time() - t0 < 0.9
+    with pytest.raises(pa.PAError, match="PA_ETIMEOUT.*device-side wait"):
+        ctx.sync_status(timeout=30.0)
+    ctx.sync_status(timeout=1.0)          # cleared; an idle stream passes at once
+    with pytest.raises(pa.PAError, match="PA_EINVAL"):
+        ctx.sync_status(timeout=-1.0)
+    wl = W.small_variant(W.workload(1), grid=(1, 20, 23), H=1, P=4, mask="all")
+    _check_case(pa, ctx, wl)
+
+
+def test_injected_allocation_failure_is_reported_and_recoverable(pa, monkeypatch):
+    # host-side injection (PA_INJECT_ENOMEM): the allocation fails as under memory
+    # pressure, the call returns PA_ENOMEM having launched nothing, and the context works
+    # again once memory is available
+    monkeypatch.setenv("PA_INJECT_ENOMEM", "init")
+    with pytest.raises(pa.PAError, match="PA_ENOMEM"):
+        pa.Context(0)
+    monkeypatch.setenv("PA_INJECT_ENOMEM", "workspace")
+    c = pa.Context(0)
+    try:
+        N, P, G, D, H = 1000, 8, 2, 128, 2
+        off = W.part_offsets(N, P)
+        fresh = np.ones((4, 4), dtype=np.uint8)
+        of, lf = _gen_states(31, P, 1, H, N, D, torch.bfloat16)
+        of, lf = of.to(DEV), lf.to(DEV)
+        o = torch.empty(1, H, N, D, dtype=torch.bfloat16, device=DEV)
+        lse = torch.full((1, H, N), float("nan"), device=DEV)
+        w = torch.full((4, P), float("nan"), device=DEV)
+        with pytest.raises(pa.PAError, match="PA_ENOMEM"):
+            pa.pa_merge_states(c, off, G, fresh, of, lf, None, None, o, lse, w)
+        with pytest.raises(pa.PAError, match="PA_ENOMEM"):
+            pa.pa_importance(c, off, G, lf, lse, w)
+        c.sync_status()
+        assert torch.isnan(lse).all() and torch.isnan(w).all()       # nothing launched
+        pa.pa_merge_states(c, off, G, fresh, of, lf, None, None, o, lse)   # no workspace needed
+        monkeypatch.delenv("PA_INJECT_ENOMEM")
+        pa.pa_merge_states(c, off, G, fresh, of, lf, None, None, o, lse, w)
+        c.sync_status()
+        ro, rl = O.merge_states(list(of.double().cpu().numpy()), list(lf.double().cpu().numpy()))
+        rw = O.importance(lf.double().cpu().numpy(), rl, off, G)
+        assert maxerr(o.float().cpu().numpy(), ro) <= TOL["bf16"]["o"]
+        assert maxerr(lse.cpu().numpy(), rl) <= TOL["bf16"]["lse"]
+        assert maxerr(w.cpu().numpy(), rw) <= TOL["bf16"]["w"]
     finally:
         c.close()
