@@ -271,6 +271,16 @@ int pa_selftest_wait(pa_ctx* ctx, double seconds, void* stream);
 int pa_relayout_seq2head(pa_ctx* ctx, const void* src, void* dst, int N, int H, int D,
                          int elem_bytes, int n_chunks, int chunk, void* stream);
 
+/* dst[h][dst_tok0 + n][:] = src[n][h][:] for n in [0, n_tok): one sequence piece,
+ * sequence-major src [n_tok][H][D], placed at its token offset in a head-major dst
+ * [H][dst_tokens][D] (dst_tok0 + n_tok <= dst_tokens).  The receive side of a chunked
+ * sequence-parallel all-to-all: each piece arriving from another rank lands in the
+ * head-major tensor attention reads -- SwiftFusion, Methodology 2 ("Torus Attention").
+ * Bit-exact; same row rules as pa_relayout_seq2head.
+ * Errors: PA_EINVAL, PA_EALIGN, PA_EUNSUPPORTED, PA_ECUDA. */
+int pa_relayout_seq2head_at(pa_ctx* ctx, const void* src, void* dst, int n_tok, int H, int D,
+                            int elem_bytes, int dst_tokens, int dst_tok0, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

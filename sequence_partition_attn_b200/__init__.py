@@ -24,6 +24,7 @@ __all__ = [
     "PA_F32", "PA_BF16", "PAError", "Context", "lib", "lib_path",
     "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head",
     "pa_merge_states_noalloc", "pa_compose_states", "pa_state_drift", "pa_selftest_wait", "EXPORTED",
+    "pa_relayout_seq2head_at",
     "select_fresh",
     "predict_fresh",
 ]
@@ -34,7 +35,8 @@ _ERRORS = {-1: "PA_EINVAL", -2: "PA_EALIGN", -3: "PA_EUNSUPPORTED", -4: "PA_ENOM
            -5: "PA_ECUDA", -6: "PA_ETIMEOUT"}
 EXPORTED = ("pa_init", "pa_destroy", "pa_last_error", "pa_sync_status", "pa_wait_status", "pa_version",
             "pa_partition_attn", "pa_merge_states", "pa_importance", "pa_relayout_seq2head",
-            "pa_merge_states_noalloc", "pa_compose_states", "pa_state_drift", "pa_selftest_wait")
+            "pa_merge_states_noalloc", "pa_compose_states", "pa_state_drift", "pa_selftest_wait",
+            "pa_relayout_seq2head_at")
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -95,11 +97,12 @@ def lib():
         L.pa_importance.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
         L.pa_compose_states.argtypes = [vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
         L.pa_relayout_seq2head.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, vp]
+        L.pa_relayout_seq2head_at.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, vp]
         L.pa_state_drift.argtypes = [vp, ci, ci, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp]
         L.pa_selftest_wait.argtypes = [vp, ctypes.c_double, vp]
         for f in ("pa_init", "pa_sync_status", "pa_wait_status", "pa_partition_attn", "pa_merge_states", "pa_merge_states_noalloc",
                   "pa_compose_states", "pa_state_drift", "pa_selftest_wait",
-                  "pa_importance", "pa_relayout_seq2head"):
+                  "pa_importance", "pa_relayout_seq2head", "pa_relayout_seq2head_at"):
             getattr(L, f).restype = ci
         _LIB = L
     return _LIB
@@ -268,6 +271,15 @@ def pa_relayout_seq2head(ctx: Context, src, dst, n_chunks=1, chunk=-1, stream=No
     _check(ctx.ptr, lib().pa_relayout_seq2head(ctx.ptr, src.data_ptr(), dst.data_ptr(), N, H, D,
                                                src.element_size(), int(n_chunks), int(chunk),
                                                _stream(stream)))
+
+
+def pa_relayout_seq2head_at(ctx: Context, src, dst, tok0, stream=None):
+    """dst[h, tok0 + n, :] = src[n, h, :]: src [n_tok, H, D] placed at token tok0 of
+    dst [H, N, D] (one piece of a chunked sequence-parallel all-to-all)."""
+    n_tok, H, D = src.shape
+    _check(ctx.ptr, lib().pa_relayout_seq2head_at(ctx.ptr, src.data_ptr(), dst.data_ptr(), n_tok, H, D,
+                                                  src.element_size(), dst.shape[-2], int(tok0),
+                                                  _stream(stream)))
 
 
 def select_fresh(w_stored, G: int, threshold: float) -> np.ndarray:

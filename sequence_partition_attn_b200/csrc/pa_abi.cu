@@ -607,8 +607,30 @@ static int pa_relayout_seq2head_impl(pa_ctx* ctx, const void* src, void* dst, in
     n0 = chunk * step < N ? chunk * step : N;
     n1 = (chunk + 1) * step < N ? (chunk + 1) * step : N;
   }
-  int e = pa::launch_relayout(src, dst, n0, n1, N, H, static_cast<int>(row_bytes), ctx->sm_count,
+  int e = pa::launch_relayout(src, dst, n0, n1, n0, N, H, static_cast<int>(row_bytes), ctx->sm_count,
                               static_cast<cudaStream_t>(stream));
+  return e ? cuda_fail(ctx, e, "relayout launch") : PA_OK;
+}
+
+static int pa_relayout_seq2head_at_impl(pa_ctx* ctx, const void* src, void* dst, int n_tok, int H, int D,
+                                        int elem_bytes, int dst_tokens, int dst_tok0, void* stream) {
+  if (!ctx) return fail(nullptr, PA_EINVAL, "ctx is NULL");
+  if (n_tok < 0 || H < 1 || D < 1) return fail(ctx, PA_EINVAL, "n_tok=%d H=%d D=%d", n_tok, H, D);
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8)
+    return fail(ctx, PA_EINVAL, "elem_bytes=%d", elem_bytes);
+  const long long row_bytes = static_cast<long long>(D) * elem_bytes;
+  if (row_bytes % 16 != 0) return fail(ctx, PA_EINVAL, "D*elem_bytes=%lld is not a multiple of 16", row_bytes);
+  if (row_bytes > 16384) return fail(ctx, PA_EUNSUPPORTED, "D*elem_bytes=%lld above 16384", row_bytes);
+  if (dst_tok0 < 0 || dst_tokens < 0 || static_cast<long long>(dst_tok0) + n_tok > dst_tokens)
+    return fail(ctx, PA_EINVAL, "tokens [%d, %lld) outside the destination's %d", dst_tok0,
+                static_cast<long long>(dst_tok0) + n_tok, dst_tokens);
+  if (n_tok == 0) return PA_OK;
+  if (!src || !dst) return fail(ctx, PA_EINVAL, "null tensor pointer");
+  if (!aligned(src, 16) || !aligned(dst, 16)) return fail(ctx, PA_EALIGN, "src and dst must be 16-byte aligned");
+  int rc = check_device(ctx);
+  if (rc) return rc;
+  int e = pa::launch_relayout(src, dst, 0, n_tok, dst_tok0, dst_tokens, H, static_cast<int>(row_bytes),
+                              ctx->sm_count, static_cast<cudaStream_t>(stream));
   return e ? cuda_fail(ctx, e, "relayout launch") : PA_OK;
 }
 
@@ -648,6 +670,12 @@ int pa_state_drift(pa_ctx* ctx, pa_dtype dtype, int B, int H, int N, int D, int 
 int pa_relayout_seq2head(pa_ctx* ctx, const void* src, void* dst, int N, int H, int D, int elem_bytes,
                          int n_chunks, int chunk, void* stream) {
   return debug_finish(ctx, stream, pa_relayout_seq2head_impl(ctx, src, dst, N, H, D, elem_bytes, n_chunks, chunk, stream));
+}
+
+int pa_relayout_seq2head_at(pa_ctx* ctx, const void* src, void* dst, int n_tok, int H, int D, int elem_bytes,
+                            int dst_tokens, int dst_tok0, void* stream) {
+  return debug_finish(ctx, stream, pa_relayout_seq2head_at_impl(ctx, src, dst, n_tok, H, D, elem_bytes, dst_tokens,
+                                                                dst_tok0, stream));
 }
 
 int pa_selftest_wait(pa_ctx* ctx, double seconds, void* stream) {

@@ -28,7 +28,8 @@ int drift_rows_per_block();
 int launch_drift(const DriftParams& prm, int dtype, int D, cudaStream_t st);
 int launch_reduce_pair(const ReducePairParams& prm, cudaStream_t st);
 
-int launch_relayout(const void* src, void* dst, long long n0, long long n1, int N, int H,
-                    int row_bytes, int sm_count, cudaStream_t st);
+// dst[h][dst_n0 + n - n0][:] = src[n][h][:], n in [n0, n1); dst has dst_N tokens per head.
+int launch_relayout(const void* src, void* dst, long long n0, long long n1, long long dst_n0, int dst_N,
+                    int H, int row_bytes, int sm_count, cudaStream_t st);
 
 }  // namespace pa

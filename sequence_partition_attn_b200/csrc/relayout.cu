@@ -3,9 +3,12 @@
 // all-to-all is cut into sequence chunks so that compute on moved chunks overlaps the
 // movement of later ones).
 //
-// dst[h][n][:] = src[n][h][:] for n in [n0, n1).  A token-head row (D * elem bytes) moves
-// whole, as 16-byte pieces: reads walk the source linearly (coalesced), writes land in
-// full contiguous rows of the destination.  Pure HBM traffic: 2 * rows * row bytes.
+// dst[h][dst_n0 + n - n0][:] = src[n][h][:] for n in [n0, n1), dst holding dst_N tokens
+// per head (the whole-sequence relayout has dst_n0 = n0 and dst_N = N; a piece of a
+// sequence-parallel all-to-all lands at its own token offset of a longer head-major
+// tensor).  A token-head row (D * elem bytes) moves whole, as 16-byte pieces: reads walk
+// the source linearly (coalesced), writes land in full contiguous rows of the
+// destination.  Pure HBM traffic: 2 * rows * row bytes.
 #include "pa_device.cuh"
 #include "pa_launch.h"
 
@@ -21,7 +24,8 @@ constexpr int kUnroll = 4;
 // kUnroll rows in flight advance by a constant step with one carry, so the loop does no
 // division.
 __global__ void __launch_bounds__(1024) relayout_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
-                                                        long long n0, long long rows, int N, int H, int ppr) {
+                                                        long long n0, long long dst_n0, long long rows, int N,
+                                                        int H, int ppr) {
   const long long gthreads = static_cast<long long>(gridDim.x) * blockDim.x;
   const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int piece = static_cast<int>(t % ppr);
@@ -38,7 +42,7 @@ __global__ void __launch_bounds__(1024) relayout_kernel(const uint4* __restrict_
     h[u] = static_cast<int>(r[u] - n[u] * H);
   }
   const uint4* s0 = src + n0 * H * ppr + piece;
-  uint4* d0 = dst + n0 * ppr + piece;
+  uint4* d0 = dst + dst_n0 * ppr + piece;
   while (r[0] < rows) {
     uint4 v[kUnroll];
 #pragma unroll
@@ -60,8 +64,8 @@ __global__ void __launch_bounds__(1024) relayout_kernel(const uint4* __restrict_
 
 }  // namespace
 
-int launch_relayout(const void* src, void* dst, long long n0, long long n1, int N, int H, int row_bytes,
-                    int sm_count, cudaStream_t st) {
+int launch_relayout(const void* src, void* dst, long long n0, long long n1, long long dst_n0, int dst_N,
+                    int H, int row_bytes, int sm_count, cudaStream_t st) {
   const int ppr = row_bytes / 16;                    // 16-byte pieces per row
   if (ppr < 1 || ppr > 1024) return static_cast<int>(cudaErrorInvalidValue);
   const int threads = ppr >= kThreads ? ppr : (kThreads / ppr) * ppr;   // a multiple of ppr
@@ -71,7 +75,7 @@ int launch_relayout(const void* src, void* dst, long long n0, long long n1, int 
   const long long cap = static_cast<long long>(sm_count) * 8;
   if (blocks > cap) blocks = cap;
   relayout_kernel<<<static_cast<unsigned>(blocks), threads, 0, st>>>(
-      static_cast<const uint4*>(src), static_cast<uint4*>(dst), n0, rows, N, H, ppr);
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), n0, dst_n0, rows, dst_N, H, ppr);
   return static_cast<int>(cudaGetLastError());
 }
 

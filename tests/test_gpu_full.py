@@ -171,16 +171,19 @@ def _run_trajectory(pa, wl, quality_heads=0, policy="threshold", margin=0.15, si
                 flips = int((mask != rmask).sum())
         err_o, err_l = maxerr(o, ro), maxerr(lse, rl)
         assert err_o <= tol["o"] and err_l <= tol["lse"], (s, err_o, err_l)
-        q_err = float("nan")
+        q_err = q_err_oracle = float("nan")
         if quality_heads:
-            # quality number: merged output against this step's fresh full attention
+            # quality numbers: the merged output (GPU, and the oracle's own reuse result on
+            # the same mask and cache) against this step's fresh full attention
             hq = slice(0, quality_heads)
             fo, fl, _ = O.partition_states(qf[:, hq], kf[:, hq], vf[:, hq], off, wl.G, ones, wl.scale)
             full_o, _ = O.merge_states(list(fo), list(fl))
             q_err = float(np.abs(o[:, hq] - full_o).max())
-        report.append((s, int(mask.sum()), err_o, err_l, q_err, flips))
+            q_err_oracle = float(np.abs(ro[:, hq] - full_o).max())
+        report.append((s, int(mask.sum()), err_o, err_l, q_err, q_err_oracle, flips))
     for r in report:
-        print("step %d fresh pairs %2d |dO| %.2e |dLSE| %.2e vs fresh full attention %.3e flips %s" % r)
+        print("step %d fresh pairs %2d |dO| %.2e |dLSE| %.2e vs fresh full attention: gpu %.3e oracle %.3e "
+              "flips %s" % r)
     ctx.close()
     return report
 
@@ -189,7 +192,7 @@ def test_denoising_trajectory_as_specified(pa):
     # threshold 0.05: with these inputs every stored importance is >= ~0.09, so no pair is
     # reused and every step is a full recompute that must still match the oracle.
     wl = W.workload(3)
-    report = _run_trajectory(pa, wl)
+    report = _run_trajectory(pa, wl, quality_heads=4)
     assert all(r[1] == wl.QG * wl.KG for r in report)
 
 

@@ -55,6 +55,25 @@ def test_relayout_bit_exact(pa, ctx, N, H, D, dt, chunks):
     assert np.array_equal(dst2.cpu().view(bits).numpy(), ref)
 
 
+@pytest.mark.parametrize("n_tok,H,D,dst_tokens,tok0,dt", [(300, 3, 128, 1000, 417, torch.bfloat16),
+                                                         (64, 2, 64, 64, 0, torch.float32),
+                                                         (7, 5, 8, 20, 13, torch.bfloat16),
+                                                         (3600, 12, 128, 115200, 57600, torch.bfloat16)])
+def test_relayout_at_places_a_piece_bit_exactly(pa, ctx, n_tok, H, D, dst_tokens, tok0, dt):
+    g = torch.Generator().manual_seed(n_tok + tok0)
+    src = torch.randn(n_tok, H, D, generator=g).to(dt)
+    bits = torch.int16 if dt == torch.bfloat16 else torch.int32
+    before = torch.randn(H, dst_tokens, D, generator=g).to(dt)
+    want = before.view(bits).numpy().copy()
+    want[:, tok0:tok0 + n_tok] = O.relayout_seq2head(src.view(bits).numpy())
+    dst = before.to(DEV)
+    pa.pa_relayout_seq2head_at(ctx, src.to(DEV), dst, tok0)
+    ctx.sync_status()
+    assert np.array_equal(dst.cpu().view(bits).numpy(), want)       # other rows untouched
+    with pytest.raises(pa.PAError, match="PA_EINVAL"):
+        pa.pa_relayout_seq2head_at(ctx, src.to(DEV), dst, dst_tokens - n_tok + 1)
+
+
 def test_relayout_rejects_rows_above_16_kib(pa, ctx):
     src = torch.zeros(4, 1, 8192, dtype=torch.float32, device=DEV)
     with pytest.raises(pa.PAError, match="PA_EUNSUPPORTED"):
