@@ -407,19 +407,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tc_fence_after();
         float s[kBN];
         {
-          uint32_t r0[32], r1[32], r2[32], r3[32];
-          tmem_ld32(tS + 0, r0);
-          tmem_ld32(tS + 32, r1);
-          tmem_ld32(tS + 64, r2);
-          tmem_ld32(tS + 96, r3);
+          uint32_t r[kBN];
+          tmem_ld128(tS, r);        // one 128-column load (fewer instructions than 4 x 32)
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            s[i] = __uint_as_float(r0[i]);
-            s[32 + i] = __uint_as_float(r1[i]);
-            s[64 + i] = __uint_as_float(r2[i]);
-            s[96 + i] = __uint_as_float(r3[i]);
-          }
+          for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(r[i]);
         }
         const int nvalid = min(kBN, k1 - key);
         if (nvalid < kBN) {
