@@ -103,35 +103,44 @@ __global__ void __launch_bounds__(kMR) merge_kernel(const __grid_constant__ Merg
   __syncthreads();
   const int nact = s_nact;
 
-  // ---- phase 1: LSE and weights, one thread per row
+  // ---- phase 1: LSE and weights, one thread per row.  The log-sum-exps are loaded eight
+  // at a time (independent loads in flight, not one latency per partition) and kept in
+  // shared memory for the weights.
   {
     const int t = threadIdx.x;
     const bool ok = t < nrows;
     float m = -INFINITY, l = 0.0f;
-    if (ok) {
-      for (int p = 0; p < P; ++p) {
-        const int e = s_state[p];
-        if (e == -1) continue;
-        const float* src = e >= 0 ? prm.lse_fresh : prm.lse_cached;
-        const float L = src[(e >= 0 ? e : -e - 2) * BHN + hrow0 + t];
+    for (int p0 = 0; p0 < P; p0 += 8) {
+      float Ls[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int p = p0 + u;
+        Ls[u] = -INFINITY;
+        if (ok && p < P) {
+          const int e = s_state[p];
+          if (e != -1) {
+            const float* src = e >= 0 ? prm.lse_fresh : prm.lse_cached;
+            Ls[u] = src[(e >= 0 ? e : -e - 2) * BHN + hrow0 + t];
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float L = Ls[u];
         if (L > m) {
           l = l * expf(m - L) + 1.0f;
           m = L;
         } else if (L > -INFINITY) {
           l += expf(L - m);
         }
+        if (p0 + u < P) sW[(p0 + u) * (kMR + 1) + t] = L;
       }
     }
     const float lse = m > -INFINITY ? m + logf(l) : -INFINITY;
     if (ok) prm.lse[hrow0 + t] = lse;
     for (int p = 0; p < P; ++p) {
-      float w = 0.0f;
-      const int e = s_state[p];
-      if (ok && lse > -INFINITY && e != -1) {
-        const float* src = e >= 0 ? prm.lse_fresh : prm.lse_cached;
-        w = expf(src[(e >= 0 ? e : -e - 2) * BHN + hrow0 + t] - lse);
-      }
-      sW[p * (kMR + 1) + t] = w;
+      const float L = sW[p * (kMR + 1) + t];
+      sW[p * (kMR + 1) + t] = (ok && lse > -INFINITY && L > -INFINITY) ? expf(L - lse) : 0.0f;
     }
   }
   __syncthreads();
@@ -143,11 +152,39 @@ __global__ void __launch_bounds__(kMR) merge_kernel(const __grid_constant__ Merg
     }
   }
 
-  // ---- phase 2: weighted sum of the state rows, one warp per row
+  // ---- phase 2: weighted sum of the state rows
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane % LPR, slot = lane / LPR;
   const uint8_t* of = static_cast<const uint8_t*>(prm.o_fresh);
   const uint8_t* oc = static_cast<const uint8_t*>(prm.o_cached);
+  if (SPW > 1 && nact <= kUnroll) {
+    // Few states per row: each group of LPR lanes takes a row of its own and loads all of
+    // its states at once, so a warp keeps SPW rows' loads in flight (no reduction across
+    // lane groups is needed: lane `sub` owns chunk `sub` of its row).
+    for (int i = warp * SPW + slot; i < nrows; i += (kMR / 32) * SPW) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const size_t rowoff = (hrow0 + i) * kRowBytes + sub * 16;
+      uint4 v[kUnroll];
+      float wt[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        wt[u] = 0.0f;
+        v[u] = make_uint4(0, 0, 0, 0);
+        if (u < nact) {
+          const int p = s_act[u];
+          const int e = s_state[p];
+          wt[u] = sW[p * (kMR + 1) + i];
+          const uint8_t* base = e >= 0 ? of : oc;
+          v[u] = __ldg(reinterpret_cast<const uint4*>(base + (e >= 0 ? e : -e - 2) * BHN * kRowBytes + rowoff));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) Acc<T>::add(acc, v[u], wt[u]);
+      *reinterpret_cast<uint4*>(static_cast<uint8_t*>(prm.o) + rowoff) = Acc<T>::pack(acc);
+    }
+    return;
+  }
+  // One warp per row.
   for (int i = warp; i < nrows; i += kMR / 32) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     const size_t rowoff = (hrow0 + i) * kRowBytes + sub * 16;
