@@ -11,9 +11,10 @@
 // both query tiles.  The running softmax restarts at each partition boundary, where the
 // epilogue writes (O_p, LSE_p).
 //
-// Roles (384 threads = 3 warpgroups, one CTA per SM, all 512 TMEM columns).  Launched at
-// 168 registers per thread; warpgroup 0 drops to 88 and the two softmax warpgroups rise to
-// 208 (88 + 2 * 208 = 3 * 168: the split uses exactly the launch allocation).
+// Roles (512 threads = 4 warpgroups, one CTA per SM, all 512 TMEM columns).  Launched at
+// 128 registers per thread; warpgroup 0 drops to 88, the epilogue warpgroup to 72 and the
+// two softmax warpgroups rise to 176 (88 + 72 + 2 * 176 = 4 * 128: the split uses exactly
+// the launch allocation).
 //   warp 0      TMA producer: Q_a and Q_b once, then K and V tiles of 128 keys into a
 //               2-stage ring.
 //   warp 1      TMEM owner and MMA issuer.  Order per KV tile j:
@@ -26,12 +27,19 @@
 //               partition end are masked, the running max is kept in the log2 domain and
 //               only moved (with a rescale of O in TMEM) when it grows by more than 8
 //               (2^8 bounds P), P is rounded to bf16 and written back over S in TMEM, and
-//               the PV product reads it from there (A operand in TMEM).
+//               the PV product reads it from there (A operand in TMEM).  At a partition's
+//               last tile the row's (max, sum) go to shared memory for the epilogue.
+//   warps 12..15 epilogue.  For each partition end, tile a then tile b: waits for the
+//               partition's last PV product and its (max, sum), reads O out of TMEM, hands
+//               O's columns back to the MMA issuer (the next partition's first PV
+//               overwrites them), and writes O_p = O / sum and LSE_p.  The softmax
+//               warpgroups never wait for these stores.
 //
 // Ordering facts the pipeline relies on: tcgen05.mma from one thread executes in issue
 // order and tcgen05.commit tracks every earlier MMA of the thread.  So the completion of
 // S_x(j+1) implies PV_x(j) is complete: the softmax may overwrite S_x / P_x columns and
-// touch O_x after waiting only for S_x(j+1).
+// touch O_x after waiting only for S_x(j+1).  The first PV product of a partition
+// (accumulate = 0) is issued only after the epilogue has read the previous partition's O.
 //
 // Exponentials run on MUFU (ex2.approx.ftz), one per score.
 #include "pa_device.cuh"
@@ -43,10 +51,12 @@ namespace {
 constexpr int kBM = 128;        // query rows per tile (MMA M)
 constexpr int kBN = 128;        // keys per tile (MMA N of S, K of PV)
 constexpr int kStages = 2;      // K/V ring depth
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kRegsLow = 88;      // warpgroup 0 (producer, MMA issuer)
-constexpr int kRegsHigh = 208;    // softmax warpgroups
-static_assert(kRegsLow + 2 * kRegsHigh == 3 * 168, "register split must equal the launch allocation");
+constexpr int kRegsEpi = 72;      // warpgroup 3 (epilogue)
+constexpr int kRegsHigh = 176;    // softmax warpgroups
+static_assert(kRegsLow + kRegsEpi + 2 * kRegsHigh == kThreads / 128 * (65536 / kThreads),
+              "register split must equal the launch allocation");
 constexpr int kAtomBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16): one swizzle-128B box
 
 template <int D>
@@ -56,10 +66,14 @@ struct Layout {
   static constexpr int kQ = 0;                             // Q_a, Q_b
   static constexpr int kK = kQ + 2 * kTileBytes;
   static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBar = kV + kStages * kTileBytes;
+  static constexpr int kML = kV + kStages * kTileBytes;     // (max, sum) per row: [tile][slot][row]
+  static constexpr int kBar = kML + 2 * 2 * kBM * 8;
+  // Per query tile x: S_FULL + x, P_LO + x, P_HI + x (softmax hand-offs), O_FINAL + x (the
+  // partition's last PV complete), ML_FULL + 2x + slot ((max, sum) of partitions of that
+  // parity written), O_FREE + x (the epilogue has read O).
   enum { Q_FULL = 0, K_FULL = 1, V_FULL = K_FULL + kStages, K_EMPTY = V_FULL + kStages,
          V_EMPTY = K_EMPTY + kStages, S_FULL = V_EMPTY + kStages, P_LO = S_FULL + 2, P_HI = P_LO + 2,
-         O_DONE = P_HI + 2, NBAR = O_DONE + 2 };
+         O_FINAL = P_HI + 2, ML_FULL = O_FINAL + 2, O_FREE = ML_FULL + 4, NBAR = O_FREE + 2 };
   static constexpr int kTmemSlot = kBar + NBAR * 8;
   static constexpr int kAbort = kTmemSlot + 8;
   static constexpr int kUsed = kAbort + 8;
@@ -192,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NBAR; ++i)
-      mbar_init(bar(i), (i >= L::P_LO && i < L::O_DONE) ? 128u : 1u);
+      mbar_init(bar(i), (i == L::O_FINAL || i == L::O_FINAL + 1) ? 1u : (i >= L::P_LO ? 128u : 1u));
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -209,7 +223,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   auto sK = [&](int s) { return base + L::kK + (uint32_t)s * L::kTileBytes; };
   auto sV = [&](int s) { return base + L::kV + (uint32_t)s * L::kTileBytes; };
 
-  if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+  // Each register change sits inside its role's branch, so that the compiler allocates
+  // every role's code under that role's own budget.
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
@@ -292,14 +309,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         int p = next_part(t, qg, 0);
         int key = t.part_off[p];
+        int e = 0;                    // ordinal of partition p among the unit's partitions
         for (; ok && j < T; ++j) {
           const bool first = key == t.part_off[p];
+          const bool last = key + kBN >= t.part_off[p + 1];
+          // A partition's first PV overwrites O_x: the epilogue must have read the last one.
+          const bool need_free = first && e > 0;
           const int s = j % kStages, s1 = (j + 1) % kStages;
           const bool more = j + 1 < T;
           const uint64_t dv = s ? dv1 : dv0;
           const uint64_t dk = s1 ? dk1 : dk0;
           // V(j) was waited for during the previous tile (or before the loop); operand
           // waits sit where products are already queued, off the hand-off path.
+          if (need_free && !wait_p(bar(L::O_FREE + 0), (e - 1) & 1)) { ok = false; break; }
           if (!wait_p(bar(L::P_LO + 0), j & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv<D, 0>(tmem + 256, tmem, dv, kIdPV, first);
@@ -312,11 +334,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (!wait_p(bar(L::P_HI + 0), j & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv<D, 1>(tmem + 256, tmem, dv, kIdPV, first);
-          commit(L::O_DONE + 0);
+          if (last) commit(L::O_FINAL + 0);
           if (more) {
             issue_s<D>(tmem, dq0, dk, kIdS);
             commit(L::S_FULL + 0);
           }
+          if (need_free && !wait_p(bar(L::O_FREE + 1), (e - 1) & 1)) { ok = false; break; }
           if (!wait_p(bar(L::P_LO + 1), j & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv<D, 0>(tmem + 384, tmem + 128, dv, kIdPV, first);
@@ -327,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (!wait_p(bar(L::P_HI + 1), j & 1)) { ok = false; break; }
           tc_fence_after();
           issue_pv<D, 1>(tmem + 384, tmem + 128, dv, kIdPV, first);
-          commit(L::O_DONE + 1);
+          if (last) commit(L::O_FINAL + 1);
           commit(L::V_EMPTY + s);
           if (more) {
             issue_s<D>(tmem + 128, dq1, dk, kIdS);
@@ -335,9 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             commit(L::K_EMPTY + s1);
           }
           key += kBN;
-          if (key >= t.part_off[p + 1]) {
+          if (last) {
             p = next_part(t, qg, p + 1);
             key = p < t.P ? t.part_off[p] : 0;
+            ++e;
           }
         }
       }
@@ -349,55 +373,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else if (warp < 12) {
     // ---------------------------------------------------------------- softmax warpgroups
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
     const int x = (warp - 4) >> 2;                 // query tile: 0 = a (warps 4-7), 1 = b
     const int wq = warp & 3;                       // TMEM lane quarter this warp may access
     const int row = wq * 32 + lane;
-    const int q_row = q_row0 + x * kBM + row;
-    const bool row_ok = q_row < q_end;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + x * 128;
     const uint32_t tO = tmem + lane_off + 256 + x * 128;
-    const size_t BHN = static_cast<size_t>(prm.BH) * prm.N;
-    __nv_bfloat16* o_part = static_cast<__nv_bfloat16*>(prm.o_part);
-
-    // Fresh partitions without keys: LSE = -inf, O = 0.
-    for (int p = 0; p < t.P; ++p) {
-      if (!fresh_bit(t.fresh_bits, qg, p) || t.part_off[p + 1] > t.part_off[p] || !row_ok) continue;
-      const size_t r = static_cast<size_t>(p) * BHN + static_cast<size_t>(bh) * prm.N + q_row;
-      uint4* dst = reinterpret_cast<uint4*>(o_part + r * D);
-      for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-      prm.lse_part[r] = -INFINITY;
-    }
-
-    auto epilogue = [&](int p, float m, float l) {
-      const float inv = 1.0f / l;
-      const size_t r = static_cast<size_t>(p) * BHN + static_cast<size_t>(bh) * prm.N + q_row;
-      uint4* dst = reinterpret_cast<uint4*>(o_part + r * D);
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tO + c * 32, v);
-        tmem_wait_ld();
-        if (row_ok) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]) * inv, __uint_as_float(v[8 * i + 1]) * inv);
-            u.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]) * inv, __uint_as_float(v[8 * i + 3]) * inv);
-            u.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]) * inv, __uint_as_float(v[8 * i + 5]) * inv);
-            u.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]) * inv, __uint_as_float(v[8 * i + 7]) * inv);
-            dst[c * 4 + i] = u;
-          }
-        }
-      }
-      if (row_ok) prm.lse_part[r] = (m + fast_log2(l)) * kLn2;
-    };
+    float2* ml_slot = reinterpret_cast<float2*>(gbase + L::kML) + (x * 2) * kBM + row;
 
     float m = -INFINITY, l = 0.0f;   // running max (log2 units, scaled) and sum
-    int j = 0, prev = -1;
+    int j = 0, e = 0;
     bool ok = true;
     const float sl2 = prm.scale_log2;
     for (int p = next_part(t, qg, 0); ok && p < t.P; p = next_part(t, qg, p + 1)) {
@@ -407,11 +396,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         tc_fence_after();
         float s[kBN];
         {
-          uint32_t r[kBN];
-          tmem_ld128(tS, r);        // one 128-column load (fewer instructions than 4 x 32)
+          uint32_t r[2][64];
+          tmem_ld64(tS, r[0]);
+          tmem_ld64(tS + 64, r[1]);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(r[i]);
+          for (int i = 0; i < kBN; ++i) s[i] = __uint_as_float(r[i >> 6][i & 63]);
         }
         const int nvalid = min(kBN, k1 - key);
         if (nvalid < kBN) {
@@ -442,8 +432,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         const float mt = row_max128(s) * sl2;
         if (key == k0) {
-          // S_x(j) complete implies PV_x(j-1) complete: O_x holds the previous partition.
-          if (prev >= 0) epilogue(prev, m, l);
           m = mt;
           l = 0.0f;
         } else if (__any_sync(0xffffffffu, mt - m > kRescaleLog2)) {
@@ -451,14 +439,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           // a row's result never depends on which rows share its warp.
           const float m_new = mt - m > kRescaleLog2 ? mt : m;
           const float alpha = fast_exp2(m - m_new);
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tO + c * 32, v);
+          // 16 columns at a time: the scores stay live here, and a narrow chunk keeps the
+          // warpgroup inside its register budget (a rescale is rare; its speed hardly matters).
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t v[16];
+            tmem_ld16(tO + c * 16, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-            tmem_st32(tO + c * 32, v);
+            for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+            tmem_st16(tO + c * 16, v);
           }
           l *= alpha;
           m = m_new;
@@ -489,12 +479,80 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const float2 a = __fadd2_rn(a01, a23);
           l += a.x + a.y;
         }
-        prev = p;
+        if (key + kBN >= k1) {
+          // The partition's last tile: its (max, sum) go to the epilogue through a slot of
+          // the partition's parity (the slot is rewritten two partitions later, after the
+          // epilogue has read it: see the ordering notes at the top).
+          ml_slot[(e & 1) * kBM] = make_float2(m, l);
+          mbar_arrive(bar(L::ML_FULL + 2 * x + (e & 1)));
+          ++e;
+        }
       }
     }
-    if (ok && j > 0 && mbar_wait(bar(L::O_DONE + x), (j - 1) & 1, abort_flag, status)) {
-      tc_fence_after();
-      epilogue(prev, m, l);
+  } else {
+    // ---------------------------------------------------------------- epilogue warpgroup
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const size_t BHN = static_cast<size_t>(prm.BH) * prm.N;
+    __nv_bfloat16* o_part = static_cast<__nv_bfloat16*>(prm.o_part);
+    const float2* ml_slot = reinterpret_cast<const float2*>(gbase + L::kML) + row;
+
+    // Fresh partitions without keys: LSE = -inf, O = 0.
+    for (int p = 0; p < t.P; ++p) {
+      if (!fresh_bit(t.fresh_bits, qg, p) || t.part_off[p + 1] > t.part_off[p]) continue;
+      for (int x = 0; x < 2; ++x) {
+        const int q_row = q_row0 + x * kBM + row;
+        if (q_row >= q_end) continue;
+        const size_t r = static_cast<size_t>(p) * BHN + static_cast<size_t>(bh) * prm.N + q_row;
+        uint4* dst = reinterpret_cast<uint4*>(o_part + r * D);
+        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+        prm.lse_part[r] = -INFINITY;
+      }
+    }
+
+    bool ok = true;
+    int e = 0;
+    for (int p = next_part(t, qg, 0); ok && p < t.P; p = next_part(t, qg, p + 1), ++e) {
+      for (int x = 0; x < 2; ++x) {
+        if (!mbar_wait(bar(L::O_FINAL + x), e & 1, abort_flag, status) ||
+            !mbar_wait(bar(L::ML_FULL + 2 * x + (e & 1)), (e >> 1) & 1, abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float2 ml = ml_slot[(x * 2 + (e & 1)) * kBM];
+        const float inv = 1.0f / ml.y;
+        const int q_row = q_row0 + x * kBM + row;
+        const bool row_ok = q_row < q_end;
+        const size_t r = static_cast<size_t>(p) * BHN + static_cast<size_t>(bh) * prm.N + q_row;
+        uint4* dst = reinterpret_cast<uint4*>(o_part + r * D);
+        const uint32_t tO = tmem + lane_off + 256 + x * 128;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tO + c * 32, v);
+          tmem_wait_ld();
+          if (c == D / 32 - 1) {
+            // O_x is out of TMEM: the issuer may start the next partition's PV into it.
+            tc_fence_before();
+            mbar_arrive(bar(L::O_FREE + x));
+          }
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 u;
+              u.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]) * inv, __uint_as_float(v[8 * i + 1]) * inv);
+              u.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]) * inv, __uint_as_float(v[8 * i + 3]) * inv);
+              u.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]) * inv, __uint_as_float(v[8 * i + 5]) * inv);
+              u.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]) * inv, __uint_as_float(v[8 * i + 7]) * inv);
+              dst[c * 4 + i] = u;
+            }
+          }
+        }
+        if (row_ok) prm.lse_part[r] = (ml.x + fast_log2(ml.y)) * kLn2;
+      }
     }
   }
 

@@ -1,7 +1,7 @@
 """The barrier protocol of the bf16 attention kernel, checked on the host.
 
-attn_tc_kernel's roles -- the TMA producer, the MMA issuer and the two softmax warpgroups --
-coordinate through mbarriers that are waited on by phase parity.  This test restates each
+attn_tc_kernel's roles -- the TMA producer, the MMA issuer, the two softmax warpgroups and the
+epilogue warpgroup -- coordinate through mbarriers that are waited on by phase parity.  This test restates each
 role's sequence of waits, arrivals and commits in program order (with the phase index
 each parity stands for), runs the roles under many random interleavings for every tile
 count up to 40, and checks that:
@@ -13,7 +13,10 @@ count up to 40, and checks that:
   reads it has been issued, an S buffer is overwritten only after the softmax has handed
   over P from it and the PV products reading that P were issued, and O is read or
   rescaled by the softmax only after the previous PV into it was issued (tcgen05 products
-  of one thread execute in issue order, and a commit tracks every earlier product).
+  of one thread execute in issue order, and a commit tracks every earlier product);
+* the epilogue reads O_x of a partition only after that partition's last PV product and
+  before the next partition's first PV product (which overwrites O_x), and reads the
+  (max, sum) slot of that partition before the softmax reuses the slot.
 
 Program order is the kernel's; MMA completion is modelled at the commit that tracks it.
 """
@@ -38,7 +41,12 @@ def producer(T):
         yield ("complete", f"V_FULL{s}")
 
 
-def issuer(T):
+def lasts_of(T, first_tiles):
+    return {j for j in range(T) if j + 1 in first_tiles or j == T - 1}
+
+
+def issuer(T, first_tiles):
+    last_tiles = lasts_of(T, first_tiles)
     yield ("wait", "Q_FULL", 0)
     if T > 0:
         yield ("wait", "K_FULL0", 0)
@@ -49,25 +57,33 @@ def issuer(T):
         yield ("complete", "S_FULL1")
         yield ("release", "K", 0)
         yield ("complete", "K_EMPTY0")
+    e = 0                                       # ordinal of the current partition
     for j in range(T):
         s, s1, more = j % STAGES, (j + 1) % STAGES, j + 1 < T
+        need_free = j in first_tiles and e > 0
+        if need_free:
+            yield ("wait", "O_FREE0", e - 1)
         yield ("wait", "P_LO0", j)
-        yield ("mma", "PVlo", 0, j)
+        yield ("mma", "PVlo", 0, j, e)
         if more:
             yield ("wait", f"K_FULL{s1}", (j + 1) // STAGES)
         yield ("wait", "P_HI0", j)
-        yield ("mma", "PVhi", 0, j)
-        yield ("complete", "O_DONE0")
+        yield ("mma", "PVhi", 0, j, e)
+        if j in last_tiles:
+            yield ("complete", "O_FINAL0")
         if more:
             yield ("mma", "S", 0, j + 1)
             yield ("complete", "S_FULL0")
+        if need_free:
+            yield ("wait", "O_FREE1", e - 1)
         yield ("wait", "P_LO1", j)
-        yield ("mma", "PVlo", 1, j)
+        yield ("mma", "PVlo", 1, j, e)
         if more:
             yield ("wait", f"V_FULL{s1}", (j + 1) // STAGES)
         yield ("wait", "P_HI1", j)
-        yield ("mma", "PVhi", 1, j)
-        yield ("complete", "O_DONE1")
+        yield ("mma", "PVhi", 1, j, e)
+        if j in last_tiles:
+            yield ("complete", "O_FINAL1")
         yield ("release", "V", j)
         yield ("complete", f"V_EMPTY{s}")
         if more:
@@ -75,26 +91,48 @@ def issuer(T):
             yield ("complete", "S_FULL1")
             yield ("release", "K", j + 1)
             yield ("complete", f"K_EMPTY{s1}")
+        if j in last_tiles:
+            e += 1
 
 
 def softmax(x, T, first_tiles):
+    last_tiles = lasts_of(T, first_tiles)
+    e = 0
     for j in range(T):
         yield ("wait", f"S_FULL{x}", j)
         yield ("read_s", x, j)
-        if j in first_tiles and j > 0:
-            yield ("touch_o", x, j)             # epilogue of the previous partition
-        yield ("touch_o", x, j)                 # a rescale may happen on any tile
+        if j not in first_tiles:
+            yield ("touch_o", x, j)             # a rescale may happen on any later tile
         yield ("write_p", x, j)
         yield ("complete", f"P_LO{x}")
         yield ("complete", f"P_HI{x}")
-    if T > 0:
-        yield ("wait", f"O_DONE{x}", T - 1)
-        yield ("touch_o", x, T)
+        if j in last_tiles:
+            yield ("write_ml", x, e)
+            yield ("complete", f"ML_FULL{x}{e & 1}")
+            e += 1
+
+
+def epilogue(T, first_tiles):
+    parts = len(first_tiles) if T > 0 else 0
+    for e in range(parts):
+        for x in range(2):
+            yield ("wait", f"O_FINAL{x}", e)
+            yield ("wait", f"ML_FULL{x}{e & 1}", e >> 1)
+            yield ("read_ml", x, e)
+            yield ("read_o", x, e)
+            yield ("complete", f"O_FREE{x}")
 
 
 class State:
-    def __init__(self, T):
+    def __init__(self, T, first_tiles):
         self.T = T
+        firsts = sorted(first_tiles)
+        self.part_first = firsts                            # partition -> first tile
+        self.part_last = [f - 1 for f in firsts[1:]] + ([T - 1] if T > 0 else [])
+        self.o_part = {0: None, 1: None}    # partition whose sums O_x accumulates
+        self.o_read = {0: -1, 1: -1}        # last partition the epilogue read out of O_x
+        self.ml_slot = {}                   # (x, slot) -> partition whose (max, sum) it holds
+        self.ml_read = {0: -1, 1: -1}
         self.done = {}                  # barrier -> completed phases
         self.loaded = {}                # ("K"|"V", stage) -> tile
         self.readers = {}               # ("K"|"V", tile) -> products issued that read it
@@ -113,17 +151,24 @@ class State:
                 need = 2 if kv == "K" else 4    # S_a, S_b read K; PV lo/hi of a and b read V
                 assert self.readers.get((kv, prev), 0) == need, f"{kv} stage {stage} reloaded early"
             self.loaded[(kv, stage)] = j
-        elif kind == "mma":
+        elif kind == "mma" and op[1] == "S":
             _, what, x, j = op
-            if what == "S":
+            if True:
                 assert self.loaded.get(("K", j % STAGES)) == j, "S issued before its K tile"
                 if self.s_tile[x] is not None:
                     assert self.p_ready[x] >= self.s_tile[x], "S overwritten before P was handed over"
                     assert self.pv_issued[x] >= self.s_tile[x], "S overwritten before PV read P"
                 self.s_tile[x] = j
                 self.readers[("K", j)] = self.readers.get(("K", j), 0) + 1
-            else:
+        elif kind == "mma":
+            _, what, x, j, e = op
+            if True:
                 assert self.loaded.get(("V", j % STAGES)) == j, "PV issued before its V tile"
+                if self.o_part[x] != e:
+                    # the first product of partition e overwrites O_x
+                    assert what == "PVlo" and j == self.part_first[e], "O_x restarted mid-partition"
+                    assert self.o_read[x] == e - 1, "O_x overwritten before the epilogue read it"
+                    self.o_part[x] = e
                 assert self.p_ready[x] >= j if what == "PVhi" else True
                 self.readers[("V", j)] = self.readers.get(("V", j), 0) + 1
                 if what == "PVhi":
@@ -138,6 +183,19 @@ class State:
         elif kind == "touch_o":
             _, x, j = op
             assert self.pv_issued[x] >= j - 1, "O touched before the previous PV was issued"
+        elif kind == "write_ml":
+            _, x, e = op
+            assert self.ml_read[x] >= e - 2, "(max, sum) slot reused before the epilogue read it"
+            self.ml_slot[(x, e & 1)] = e
+        elif kind == "read_ml":
+            _, x, e = op
+            assert self.ml_slot.get((x, e & 1)) == e, "epilogue read another partition's (max, sum)"
+            self.ml_read[x] = e
+        elif kind == "read_o":
+            _, x, e = op
+            assert self.o_part[x] == e, "epilogue read O of another partition"
+            assert self.pv_issued[x] == self.part_last[e], "epilogue read O before its last PV"
+            self.o_read[x] = e
 
 
 def runnable(st, op):
@@ -152,9 +210,10 @@ def runnable(st, op):
 
 def simulate(T, first_tiles, seed):
     rng = random.Random(seed)
-    st = State(T)
-    roles = {"producer": producer(T), "issuer": issuer(T),
-             "softmax0": softmax(0, T, first_tiles), "softmax1": softmax(1, T, first_tiles)}
+    st = State(T, first_tiles)
+    roles = {"producer": producer(T), "issuer": issuer(T, first_tiles),
+             "softmax0": softmax(0, T, first_tiles), "softmax1": softmax(1, T, first_tiles),
+             "epilogue": epilogue(T, first_tiles)}
     pending = {name: next(g, None) for name, g in roles.items()}
     while any(op is not None for op in pending.values()):
         ready = [n for n, op in pending.items() if op is not None and runnable(st, op)]
@@ -172,7 +231,7 @@ def simulate(T, first_tiles, seed):
 def test_attention_pipeline_protocol(T):
     rng = random.Random(T)
     for seed in range(25):
-        # partitions of 1..5 tiles: their first tiles trigger the epilogue
+        # partitions of 1..5 tiles; each partition end goes through the epilogue
         firsts, j = set(), 0
         while j < T:
             firsts.add(j)
