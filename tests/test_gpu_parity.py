@@ -209,6 +209,36 @@ def test_bf16_maximum_partition_count(pa, ctx):
     _check_case(pa, ctx, wl, fresh)
 
 
+def _units(wl, fresh):
+    """Work units of the bf16 launch: 256-row blocks of query groups with a fresh pair."""
+    rb = W.group_row_bounds(W.part_offsets(wl.N, wl.P), wl.G)
+    return wl.B * wl.H * sum(-(-(int(rb[g + 1]) - int(rb[g])) // 256)
+                             for g in range(wl.QG) if fresh[g].any() and rb[g + 1] > rb[g])
+
+
+def test_bf16_many_units_ragged(pa, ctx):
+    # More work units (CTAs) than SMs, 200-key partitions (a shifted last tile each) and a
+    # random mask.
+    wl = W.small_variant(W.workload(1), grid=(1, 30, 40), H=40, P=6, G=1)
+    fresh = (np.random.default_rng(5).random((wl.QG, wl.KG)) < 0.5).astype(np.uint8)
+    np.fill_diagonal(fresh, 1)
+    assert _units(wl, fresh) > 148
+    _check_case(pa, ctx, wl, fresh)
+
+
+def test_bf16_units_of_short_partitions(pa, ctx):
+    # More units than SMs, each of partitions shorter than a tile (4 keys), an empty
+    # partition, a query group whose only fresh partition is the empty one (a unit without
+    # KV tiles: it only writes LSE = -inf, O = 0) and an idle query group; D = 64.
+    wl = W.small_variant(W.workload(1), grid=(1, 4, 4), H=64, P=5, G=1, D=64)
+    fresh = (np.random.default_rng(9).random((wl.QG, wl.KG)) < 0.6).astype(np.uint8)
+    fresh[0] = 1
+    fresh[3] = [0, 0, 0, 0, 1]
+    fresh[1] = 0
+    assert _units(wl, fresh) > 148
+    _check_case(pa, ctx, wl, fresh)
+
+
 def test_fp32_small_ragged_case(pa, ctx):
     wl = W.small_variant(W.workload(0), grid=(1, 13, 23), H=2, P=3, G=1, cache_sigma=0.05,
                          mask="neighbours", D=128)

@@ -16,9 +16,13 @@ count up to 40, and checks that:
   of one thread execute in issue order, and a commit tracks every earlier product);
 * the epilogue reads O_x of a partition only after that partition's last PV product and
   before the next partition's first PV product (which overwrites O_x), and reads the
-  (max, sum) slot of that partition before the softmax reuses the slot.
+  (max, sum) slot of that partition before the softmax reuses the slot;
+* no product reads a Q, K or V tile before its load has landed.
 
-Program order is the kernel's; MMA completion is modelled at the commit that tracks it.
+A CTA's work is a list of partition lengths in KV tiles.
+
+Program order is the kernel's; MMA completion is modelled at the commit that tracks it.  A
+TMA load completes (lands and arrives on its barrier) at any later step, in any order.
 """
 import random
 
@@ -27,36 +31,43 @@ import pytest
 STAGES = 2
 
 
-def producer(T):
-    yield ("complete", "Q_FULL")
-    for j in range(T):
+class Work:
+    """Tile structure of a CTA's work: parts = [tiles of each partition]."""
+
+    def __init__(self, parts):
+        self.T = sum(parts)
+        self.first_tiles, j = set(), 0
+        for n in parts:
+            self.first_tiles.add(j)
+            j += n
+        self.last_tiles = {j for j in range(self.T) if j + 1 in self.first_tiles or j == self.T - 1}
+
+
+def producer(w):
+    yield ("tma", ("Q",), "Q_FULL")             # Q_a and Q_b, one barrier
+    for j in range(w.T):
         s = j % STAGES
         if j >= STAGES:
             yield ("wait", f"K_EMPTY{s}", j // STAGES - 1)
-        yield ("load", "K", j)
-        yield ("complete", f"K_FULL{s}")
+        yield ("tma", ("K", j), f"K_FULL{s}")
         if j >= STAGES:
             yield ("wait", f"V_EMPTY{s}", j // STAGES - 1)
-        yield ("load", "V", j)
-        yield ("complete", f"V_FULL{s}")
+        yield ("tma", ("V", j), f"V_FULL{s}")
 
 
-def lasts_of(T, first_tiles):
-    return {j for j in range(T) if j + 1 in first_tiles or j == T - 1}
-
-
-def issuer(T, first_tiles):
-    last_tiles = lasts_of(T, first_tiles)
+def issuer(w):
+    T, first_tiles, last_tiles = w.T, w.first_tiles, w.last_tiles
     yield ("wait", "Q_FULL", 0)
-    if T > 0:
-        yield ("wait", "K_FULL0", 0)
-        yield ("wait", "V_FULL0", 0)
-        yield ("mma", "S", 0, 0)
-        yield ("complete", "S_FULL0")
-        yield ("mma", "S", 1, 0)
-        yield ("complete", "S_FULL1")
-        yield ("release", "K", 0)
-        yield ("complete", "K_EMPTY0")
+    if T == 0:
+        return
+    yield ("wait", "K_FULL0", 0)
+    yield ("wait", "V_FULL0", 0)
+    yield ("mma", "S", 0, 0)
+    yield ("complete", "S_FULL0")
+    yield ("mma", "S", 1, 0)
+    yield ("complete", "S_FULL1")
+    yield ("release", "K", 0)
+    yield ("complete", "K_EMPTY0")
     e = 0                                       # ordinal of the current partition
     for j in range(T):
         s, s1, more = j % STAGES, (j + 1) % STAGES, j + 1 < T
@@ -95,8 +106,8 @@ def issuer(T, first_tiles):
             e += 1
 
 
-def softmax(x, T, first_tiles):
-    last_tiles = lasts_of(T, first_tiles)
+def softmax(x, w):
+    T, first_tiles, last_tiles = w.T, w.first_tiles, w.last_tiles
     e = 0
     for j in range(T):
         yield ("wait", f"S_FULL{x}", j)
@@ -112,9 +123,8 @@ def softmax(x, T, first_tiles):
             e += 1
 
 
-def epilogue(T, first_tiles):
-    parts = len(first_tiles) if T > 0 else 0
-    for e in range(parts):
+def epilogue(w):
+    for e in range(len(w.first_tiles)):
         for x in range(2):
             yield ("wait", f"O_FINAL{x}", e)
             yield ("wait", f"ML_FULL{x}{e & 1}", e >> 1)
@@ -124,9 +134,11 @@ def epilogue(T, first_tiles):
 
 
 class State:
-    def __init__(self, T, first_tiles):
+    def __init__(self, w):
+        T = w.T
         self.T = T
-        firsts = sorted(first_tiles)
+        self.w = w
+        firsts = sorted(w.first_tiles)
         self.part_first = firsts                            # partition -> first tile
         self.part_last = [f - 1 for f in firsts[1:]] + ([T - 1] if T > 0 else [])
         self.o_part = {0: None, 1: None}    # partition whose sums O_x accumulates
@@ -135,6 +147,7 @@ class State:
         self.ml_read = {0: -1, 1: -1}
         self.done = {}                  # barrier -> completed phases
         self.loaded = {}                # ("K"|"V", stage) -> tile
+        self.landed = set()             # loads whose data has arrived
         self.readers = {}               # ("K"|"V", tile) -> products issued that read it
         self.s_tile = {0: None, 1: None}    # tile whose scores the S buffer holds
         self.p_ready = {0: -1, 1: -1}       # last tile whose P was handed over
@@ -143,8 +156,8 @@ class State:
 
     def check(self, op, role):
         kind = op[0]
-        if kind == "load":
-            _, kv, j = op
+        if kind == "tma" and op[1][0] in "KV":
+            _, (kv, j), _ = op
             stage = j % STAGES
             prev = self.loaded.get((kv, stage))
             if prev is not None:
@@ -153,26 +166,27 @@ class State:
             self.loaded[(kv, stage)] = j
         elif kind == "mma" and op[1] == "S":
             _, what, x, j = op
-            if True:
-                assert self.loaded.get(("K", j % STAGES)) == j, "S issued before its K tile"
-                if self.s_tile[x] is not None:
-                    assert self.p_ready[x] >= self.s_tile[x], "S overwritten before P was handed over"
-                    assert self.pv_issued[x] >= self.s_tile[x], "S overwritten before PV read P"
-                self.s_tile[x] = j
-                self.readers[("K", j)] = self.readers.get(("K", j), 0) + 1
+            assert ("Q",) in self.landed, "score product issued before Q landed"
+            assert ("K", j) in self.landed, "score product issued before its K tile landed"
+            assert self.loaded.get(("K", j % STAGES)) == j, "S issued before its K tile"
+            if self.s_tile[x] is not None:
+                assert self.p_ready[x] >= self.s_tile[x], "S overwritten before P was handed over"
+                assert self.pv_issued[x] >= self.s_tile[x], "S overwritten before PV read P"
+            self.s_tile[x] = j
+            self.readers[("K", j)] = self.readers.get(("K", j), 0) + 1
         elif kind == "mma":
             _, what, x, j, e = op
-            if True:
-                assert self.loaded.get(("V", j % STAGES)) == j, "PV issued before its V tile"
-                if self.o_part[x] != e:
-                    # the first product of partition e overwrites O_x
-                    assert what == "PVlo" and j == self.part_first[e], "O_x restarted mid-partition"
-                    assert self.o_read[x] == e - 1, "O_x overwritten before the epilogue read it"
-                    self.o_part[x] = e
-                assert self.p_ready[x] >= j if what == "PVhi" else True
-                self.readers[("V", j)] = self.readers.get(("V", j), 0) + 1
-                if what == "PVhi":
-                    self.pv_issued[x] = j
+            assert self.loaded.get(("V", j % STAGES)) == j, "PV issued before its V tile"
+            assert ("V", j) in self.landed, "PV issued before its V tile landed"
+            if self.o_part[x] != e:
+                # the first product of partition e overwrites O_x
+                assert what == "PVlo" and j == self.part_first[e], "O_x restarted mid-partition"
+                assert self.o_read[x] == e - 1, "O_x overwritten before the epilogue read it"
+                self.o_part[x] = e
+            assert self.p_ready[x] >= j if what == "PVhi" else True
+            self.readers[("V", j)] = self.readers.get(("V", j), 0) + 1
+            if what == "PVhi":
+                self.pv_issued[x] = j
         elif kind == "read_s":
             _, x, j = op
             assert self.s_tile[x] == j, "softmax read a score buffer holding another tile"
@@ -208,32 +222,48 @@ def runnable(st, op):
     return c > k
 
 
-def simulate(T, first_tiles, seed):
+def simulate(parts, seed):
     rng = random.Random(seed)
-    st = State(T, first_tiles)
-    roles = {"producer": producer(T), "issuer": issuer(T, first_tiles),
-             "softmax0": softmax(0, T, first_tiles), "softmax1": softmax(1, T, first_tiles),
-             "epilogue": epilogue(T, first_tiles)}
+    w = Work(parts)
+    T = w.T
+    st = State(w)
+    roles = {"producer": producer(w), "issuer": issuer(w),
+             "softmax0": softmax(0, w), "softmax1": softmax(1, w), "epilogue": epilogue(w)}
     pending = {name: next(g, None) for name, g in roles.items()}
-    while any(op is not None for op in pending.values()):
+    in_flight = []                      # issued TMA loads: (what, barrier)
+    land_p = (0.01, 0.1, 0.5)[seed % 3]   # slow loads stay in flight across many steps
+    while any(op is not None for op in pending.values()) or in_flight:
         ready = [n for n, op in pending.items() if op is not None and runnable(st, op)]
-        assert ready, f"deadlock at T={T}: " + str({n: op for n, op in pending.items() if op})
+        assert ready or in_flight, f"deadlock at T={T}: " + str({n: op for n, op in pending.items() if op})
+        if in_flight and (not ready or rng.random() < land_p):
+            # a load lands (any of those in flight) and arrives on its barrier
+            what, bar = in_flight.pop(rng.randrange(len(in_flight)))
+            st.landed.add(what)
+            st.done[bar] = st.done.get(bar, 0) + 1
+            continue
         name = rng.choice(ready)
         op = pending[name]
         if op[0] == "complete":
             st.done[op[1]] = st.done.get(op[1], 0) + 1
         else:
             st.check(op, name)
+            if op[0] == "tma":
+                in_flight.append((op[1], op[2]))
         pending[name] = next(roles[name], None)
+
+
+def _partitions(rng, T):
+    parts, j = [], 0
+    while j < T:
+        n = min(rng.randint(1, 5), T - j)
+        parts.append(n)
+        j += n
+    return parts
 
 
 @pytest.mark.parametrize("T", list(range(0, 41)))
 def test_attention_pipeline_protocol(T):
+    # partitions of 1..5 tiles, each partition end going through the epilogue
     rng = random.Random(T)
     for seed in range(25):
-        # partitions of 1..5 tiles; each partition end goes through the epilogue
-        firsts, j = set(), 0
-        while j < T:
-            firsts.add(j)
-            j += rng.randint(1, 5)
-        simulate(T, firsts, seed)
+        simulate(_partitions(rng, T), seed)
