@@ -182,7 +182,7 @@ __device__ __forceinline__ void exp_pack_half(const float (&s)[128], float m, fl
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams prm) {
+__device__ __forceinline__ void attn_tc_body(const TcParams& prm, const int unit) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -197,8 +197,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int lane = threadIdx.x & 31;
 
   // Decode the work unit: (b*H + h, query group, 256-row block of the group).
-  const int bh = blockIdx.x / prm.tiles_total;
-  const int tix = blockIdx.x - bh * prm.tiles_total;
+  const int bh = unit / prm.tiles_total;
+  const int tix = unit - bh * prm.tiles_total;
   int qg = 0;
   while (qg + 1 < t.QG && t.tile_start[qg + 1] <= tix) ++qg;
   const int q_row0 = t.qg_row0[qg] + (tix - t.tile_start[qg]) * (2 * kBM);
@@ -564,19 +564,38 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   }
 }
 
+// One CTA per work unit.  Unit = blockIdx.x; or, for a grid of a few waves, the unit that
+// the host's longest-first order puts at that position: the hardware hands out CTAs in
+// blockIdx order as SMs free up, so the longest units start first and the last wave holds
+// the shortest ones (a shorter tail when units differ in length).
 template <int D>
-int launch_impl(const TcParams& prm, int units, cudaStream_t st) {
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams prm) {
+  attn_tc_body<D>(prm, static_cast<int>(blockIdx.x));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_ordered_kernel(const __grid_constant__ TcParams prm,
+                                                                      const __grid_constant__ TcUnitOrder ord) {
+  attn_tc_body<D>(prm, static_cast<int>(ord.unit[blockIdx.x]));
+}
+
+template <int D>
+int launch_impl(const TcParams& prm, const TcUnitOrder* ord, int units, cudaStream_t st) {
   const int smem = Layout<D>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = ord ? cudaFuncSetAttribute(attn_tc_ordered_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                      : cudaFuncSetAttribute(attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return static_cast<int>(e);
-  attn_tc_kernel<D><<<units, kThreads, smem, st>>>(prm);
+  if (ord)
+    attn_tc_ordered_kernel<D><<<units, kThreads, smem, st>>>(prm, *ord);
+  else
+    attn_tc_kernel<D><<<units, kThreads, smem, st>>>(prm);
   return static_cast<int>(cudaGetLastError());
 }
 
 }  // namespace
 
-int launch_attn_tc(const TcParams& prm, int units, cudaStream_t st) {
-  return prm.D == 64 ? launch_impl<64>(prm, units, st) : launch_impl<128>(prm, units, st);
+int launch_attn_tc(const TcParams& prm, const TcUnitOrder* ord, int units, cudaStream_t st) {
+  return prm.D == 64 ? launch_impl<64>(prm, ord, units, st) : launch_impl<128>(prm, ord, units, st);
 }
 
 // Query rows per work unit (two 128-row tiles).

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <chrono>
 #include <cstdarg>
 #include <cstdlib>
@@ -11,6 +12,8 @@
 #include <mutex>
 #include <string>
 #include <thread>
+#include <utility>
+#include <vector>
 
 #include "../../include/pa.h"
 #include "pa_device.cuh"
@@ -119,6 +122,36 @@ int fill_tile_start(pa::AttnTables& t, int tile_rows) {
   }
   t.tile_start[t.QG] = acc;
   return acc;
+}
+
+// Longest-first launch order for a bf16 attention grid of a few waves (more units than SMs,
+// at most kMaxOrderedUnits): units sorted by their KV tile count, longest first, ties in
+// unit order (stable).  Returns false, and leaves the grid in unit order, when every unit
+// has the same length or the grid is one wave or very large: there the order cannot shorten
+// the tail, and unit order keeps the CTAs of one head (which share K and V) together.
+bool longest_first(const pa::TcParams& prm, int units, int sm_count, pa::TcUnitOrder& ord) {
+  if (units <= sm_count || units > pa::kMaxOrderedUnits) return false;
+  const pa::AttnTables& t = prm.t;
+  int group_tiles[PA_MAX_P];
+  for (int qg = 0; qg < t.QG; ++qg) {
+    group_tiles[qg] = 0;
+    for (int p = 0; p < t.P; ++p)
+      if (pa::fresh_bit(t.fresh_bits, qg, p) && t.part_off[p + 1] > t.part_off[p])
+        group_tiles[qg] += (t.part_off[p + 1] - t.part_off[p] + 127) / 128;
+  }
+  std::vector<std::pair<int, int>> key(units);        // (-tiles, unit)
+  bool varied = false;
+  for (int u = 0; u < units; ++u) {
+    const int tix = u % prm.tiles_total;
+    int qg = 0;
+    while (qg + 1 < t.QG && t.tile_start[qg + 1] <= tix) ++qg;
+    key[u] = {-group_tiles[qg], u};
+    varied |= key[u].first != key[0].first;
+  }
+  if (!varied) return false;
+  std::stable_sort(key.begin(), key.end());
+  for (int i = 0; i < units; ++i) ord.unit[i] = static_cast<uint16_t>(key[i].second);
+  return true;
 }
 
 // Host-side fault injection for tests (no GPU fault involved): PA_INJECT_ENOMEM, a
@@ -400,7 +433,9 @@ static int pa_partition_attn_impl(pa_ctx* ctx, const pa_attn_desc* d, void* stre
     prm.scale_log2 = d->scale * 1.4426950408889634f;
     const long long units = BH * tiles;
     if (units > 0x7fffffffLL) return fail(ctx, PA_EINVAL, "too many work units");
-    int e = pa::launch_attn_tc(prm, static_cast<int>(units), st);
+    pa::TcUnitOrder order;
+    const bool ordered = longest_first(prm, static_cast<int>(units), ctx->sm_count, order);
+    int e = pa::launch_attn_tc(prm, ordered ? &order : nullptr, static_cast<int>(units), st);
     return e ? cuda_fail(ctx, e, "attn_tc launch") : PA_OK;
   }
   pa::F32AttnParams prm;

@@ -32,6 +32,13 @@ struct TcParams {
   AttnTables t;
 };
 
+// Launch order of the work units of a bf16 attention grid of a few waves: CTA i processes
+// unit unit[i] (a permutation of 0 .. units - 1, longest units first).
+constexpr int kMaxOrderedUnits = 2048;
+struct TcUnitOrder {
+  uint16_t unit[kMaxOrderedUnits];
+};
+
 struct F32AttnParams {
   const float* q;
   const float* k;

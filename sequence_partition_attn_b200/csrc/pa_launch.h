@@ -8,7 +8,8 @@
 
 namespace pa {
 
-int launch_attn_tc(const TcParams& prm, int units, cudaStream_t st);
+// One CTA per work unit: CTA i takes unit i, or unit ord->unit[i] when `ord` is given.
+int launch_attn_tc(const TcParams& prm, const TcUnitOrder* ord, int units, cudaStream_t st);
 int attn_tc_tile_rows();
 
 int launch_attn_f32(const F32AttnParams& prm, cudaStream_t st);
