@@ -72,7 +72,9 @@ int launch_relayout(const void* src, void* dst, long long n0, long long n1, long
   const long long rows = (n1 - n0) * H;
   if (rows <= 0) return 0;
   long long blocks = (rows * ppr + static_cast<long long>(threads) * kUnroll - 1) / (static_cast<long long>(threads) * kUnroll);
-  const long long cap = static_cast<long long>(sm_count) * 8;
+  // up to 32 blocks per SM (8 resident at once): the grid-stride loop then ends more evenly
+  // (228 / 233 / 242 us on [115200][24][128] bf16 with 32 / 16 / 8 per SM)
+  const long long cap = static_cast<long long>(sm_count) * 32;
   if (blocks > cap) blocks = cap;
   relayout_kernel<<<static_cast<unsigned>(blocks), threads, 0, st>>>(
       static_cast<const uint4*>(src), static_cast<uint4*>(dst), n0, dst_n0, rows, dst_N, H, ppr);
