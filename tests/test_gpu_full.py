@@ -25,12 +25,14 @@ def pa():
 
 
 def _rows_720p(wl):
+    # 512 random rows, the first two 128-row query tiles of the first query partition, the
+    # last 256 rows (the ragged last partition) and a query-group boundary, on every head
     off = W.part_offsets(wl.N, wl.P)
     rng = np.random.default_rng(11)
-    r = rng.choice(wl.N, size=64, replace=False)
-    first = np.arange(0, 24)
-    tail = np.arange(off[-1] - 40, off[-1])                    # ragged last partition
-    bound = np.arange(off[4] - 8, off[4] + 8)                  # a query-group boundary
+    r = rng.choice(wl.N, size=512, replace=False)
+    first = np.arange(0, 256)
+    tail = np.arange(off[-1] - 256, off[-1])
+    bound = np.arange(off[4] - 8, off[4] + 8)
     return np.unique(np.concatenate([r, first, tail, bound]))
 
 
@@ -262,8 +264,10 @@ def test_ulysses_layout_full_size(pa):
     ctx.sync_status()
     assert torch.equal(l_ov, l_seq) and torch.equal(o_ov.view(torch.int16), o_seq.view(torch.int16))
     del o_seq, l_seq, o_ov, l_ov
-    rows = np.unique(np.concatenate([np.random.default_rng(4).choice(N, 48, replace=False),
-                                     np.arange(7200 - 4, 7200 + 4), np.arange(N - 8, N)]))
+    # 512 random rows, the first and last 256 rows and a chunk boundary, on every head
+    rows = np.unique(np.concatenate([np.random.default_rng(4).choice(N, 512, replace=False),
+                                     np.arange(0, 256), np.arange(7200 - 4, 7200 + 4),
+                                     np.arange(N - 256, N)]))
     ri = torch.as_tensor(rows, device=DEV)
     go = o.index_select(2, ri).float().cpu().numpy()
     gl = lse.index_select(2, ri).cpu().numpy()
