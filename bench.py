@@ -328,6 +328,49 @@ def config_extras(ctx, dev, stream, pk, reps=20):
                       "attention_ms": ms, "attention_tflops": fl / (ms / 1e3) / 1e12,
                       "attention_frac_of_burst": fl / (ms / 1e3) / 1e12 / pk["bf16_tflops"]}
     del q, k, v, o, lse, flush
+    out["config3"] = trajectory_extras(ctx, dev, stream, pk)
+    return out
+
+
+def trajectory_extras(ctx, dev, stream, pk):
+    """The denoising trajectory (image-DiT shape, 10 steps, K and V drifting, anchors 0 and 5)
+    under each reuse policy: the threshold as specified (0.05), a threshold that reuses
+    (0.12) and the online prediction.  Per step, wall time on the host around the step
+    (device work, the host's mask selection, and at anchors the copy of w to the host) with
+    the stream synchronized on both sides; inputs of every step are generated and moved to
+    the device before timing."""
+    from sequence_partition_attn_b200.step import Trajectory
+    wl = W.workload(3)
+    off = W.part_offsets(wl.N, wl.P)
+    host = W.make_qkv(wl)
+    q = host["q"].to(dev)
+    kv, k, v = [], host["k"], host["v"]
+    for s_ in range(wl.steps):
+        if s_ > 0:
+            k, v = W.drift_kv(wl, k, v, s_)
+        kv.append((k.to(dev), v.to(dev)))
+    per_pair = 4.0 * wl.D * wl.B * wl.H * float(wl.N // wl.P) ** 2     # flops of one (query, KV) partition pair
+    out = {"workload": f"{wl.name}: B{wl.B} H{wl.H} N{wl.N} D{wl.D} bf16, P={wl.P}, {wl.steps} steps, "
+                       f"anchors {list(wl.anchors)}, drift {wl.drift}"}
+    for name, thr, policy in (("threshold_0.05", wl.threshold, "threshold"), ("threshold_0.12", 0.12, "threshold"),
+                              ("online_prediction", 1e-3, "predict")):
+        tr = Trajectory(ctx, wl.B, wl.H, wl.N, wl.D, off, wl.G, wl.anchors, thr, device=dev, policy=policy)
+        times, fresh = [], []
+        for s_ in range(wl.steps):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            mask = tr.step(s_, q, kv[s_][0], kv[s_][1], stream=stream)
+            torch.cuda.synchronize()
+            times.append((time.perf_counter() - t0) * 1e3)
+            fresh.append(int(mask.sum()))
+        ctx.sync_status()
+        reuse_steps = [i for i in range(wl.steps) if i not in wl.anchors]
+        out[name] = {"ms_per_step": times, "fresh_pairs_per_step": fresh, "pairs": int(wl.P * wl.P),
+                     "mean_ms_anchor": statistics.mean(times[i] for i in wl.anchors),
+                     "mean_ms_between_anchors": statistics.mean(times[i] for i in reuse_steps),
+                     "attention_flops_per_step": [f * per_pair for f in fresh]}
+        del tr
+    del kv, q
     return out
 
 
